@@ -1,0 +1,258 @@
+"""Python binding of libblasst.so (BLASST blocked attention on B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/blasst.h``.  PyTorch supplies
+device memory and streams.  There is no CPU fallback: if the shared library
+is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "BlasstError", "lib", "prefill", "decode", "calibrate", "calibrate_fit", "calibrate_threshold",
+    "visited_pairs", "decode_workspace_bytes", "mask_words", "Opts", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libblasst.so")
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace too small",
+          4: "CUDA error", 5: "device wait timed out"}
+
+
+class BlasstError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        msg = f"{what}: {STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class Opts(ctypes.Structure):
+    """Mirror of ``blasst_opts``."""
+
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("dv", ctypes.c_int),
+        ("block_n", ctypes.c_int),
+        ("num_splits", ctypes.c_int),
+        ("mode", ctypes.c_int),
+        ("k_row_stride", ctypes.c_longlong),
+        ("v_row_stride", ctypes.c_longlong),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("gaps_out", ctypes.c_void_p),
+        ("status_word", ctypes.c_void_p),
+    ]
+
+    def __init__(self, **kw):
+        super().__init__()
+        self.struct_size = ctypes.sizeof(Opts)
+        for k, v in kw.items():
+            setattr(self, k, v)
+
+
+_ATTN_ARGS = [ctypes.c_void_p] * 4 + [ctypes.c_void_p] + [ctypes.c_int] * 6 + [ctypes.c_float, ctypes.c_float,
+                                                                              ctypes.c_int, ctypes.c_void_p,
+                                                                              ctypes.c_void_p, ctypes.c_void_p,
+                                                                              ctypes.POINTER(Opts)]
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libblasst.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m block_sparse_flashattention_tcgen05_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name in ("blasst_prefill", "blasst_decode", "blasst_calibrate"):
+            f = getattr(L, name)
+            f.restype = ctypes.c_int
+            f.argtypes = _ATTN_ARGS
+        L.blasst_calibrate_fit.restype = ctypes.c_int
+        L.blasst_calibrate_fit.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                                                                   ctypes.POINTER(ctypes.c_double)]
+        L.blasst_calibrate_threshold.restype = ctypes.c_int
+        L.blasst_calibrate_threshold.argtypes = [ctypes.c_void_p, ctypes.c_longlong, ctypes.c_double,
+                                                 ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+        L.blasst_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.blasst_decode_workspace_bytes.argtypes = [ctypes.c_int] * 5
+        L.blasst_visited_pairs.restype = ctypes.c_longlong
+        L.blasst_visited_pairs.argtypes = [ctypes.c_int] * 7 + [ctypes.POINTER(Opts)]
+        L.blasst_status_string.restype = ctypes.c_char_p
+        L.blasst_status_string.argtypes = [ctypes.c_int]
+        L.blasst_last_error.restype = ctypes.c_char_p
+        L.blasst_last_error.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        detail = lib().blasst_last_error().decode() if rc == 4 else ""
+        raise BlasstError(rc, what, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def mask_words(n_blocks: int) -> int:
+    return (n_blocks + 31) // 32
+
+
+def _dev_tensor(t, name):
+    import torch
+
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers)")
+    return t
+
+
+def _attn(fn_name, q, k, v, *, scale, lam, causal, o, lse, want_mask, want_count, opts, stream, mask_rows,
+          n_blocks, B, Hq, Hkv, Lq, Lk, d, dv):
+    import torch
+
+    dev = q.device
+    if want_mask is True:
+        want_mask = torch.empty((mask_rows, mask_words(n_blocks)), dtype=torch.int32, device=dev)
+    if want_count is True:
+        want_count = torch.empty(1, dtype=torch.int64, device=dev)
+    mask = want_mask if isinstance(want_mask, torch.Tensor) else None
+    count = want_count if isinstance(want_count, torch.Tensor) else None
+    rc = getattr(lib(), fn_name)(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, d, float(scale), float(lam),
+        int(bool(causal)), _ptr(mask), _ptr(count), _stream(stream), ctypes.byref(opts))
+    _check(rc, fn_name)
+    return mask, count
+
+
+def prefill(q, k, v, *, scale, lam=0.0, causal=True, o=None, lse=None, skip_mask=True, skip_count=True,
+            status_word=None, stream=None):
+    """Prefill attention with block skipping.  q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA.
+
+    Returns (o, lse, skip_mask [B*Hq*ceil(Lq/128), W] int32 or None, skip_count [1] int64 or None).
+    """
+    import torch
+
+    _dev_tensor(q, "q"), _dev_tensor(k, "k"), _dev_tensor(v, "v")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if o is None:
+        o = torch.empty((B, Hq, Lq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    opts = Opts(status_word=None if status_word is None else status_word.data_ptr())
+    nq = (Lq + 127) // 128
+    nb = (Lk + 127) // 128
+    m, c = _attn("blasst_prefill", q, k, v, scale=scale, lam=lam, causal=causal, o=o, lse=lse,
+                 want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hq * nq,
+                 n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=d)
+    return o, lse, m, c
+
+
+def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=None, skip_mask=True,
+           skip_count=True, workspace=None, status_word=None, stream=None):
+    """Split-KV decode with block skipping.  q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA.
+
+    Returns (o, lse, skip_mask [B*Hkv, W] int32 or None, skip_count [1] int64 or None).
+    ``workspace``: optional uint8 CUDA tensor of at least decode_workspace_bytes() bytes.
+    """
+    import torch
+
+    _dev_tensor(q, "q"), _dev_tensor(k, "k"), _dev_tensor(v, "v")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    opts = Opts(num_splits=num_splits, dv=dv,
+                status_word=None if status_word is None else status_word.data_ptr())
+    if workspace is not None:
+        opts.workspace = workspace.data_ptr()
+        opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    nb = (Lk + 63) // 64
+    m, c = _attn("blasst_decode", q, k, v, scale=scale, lam=lam, causal=causal, o=o, lse=lse,
+                 want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hkv,
+                 n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=dv)
+    return o, lse, m, c
+
+
+def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=16, skip_mask=True,
+              skip_count=True, stream=None):
+    """Decision-only pass.  Returns (gaps [tiles, nb] fp32, skip_mask, skip_count)."""
+    import torch
+
+    _dev_tensor(q, "q"), _dev_tensor(k, "k")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if mode == "prefill":
+        nb = (Lk + 127) // 128
+        tiles = B * Hq * ((Lq + 127) // 128)
+        m = 0
+    elif mode == "decode":
+        nb = (Lk + 63) // 64
+        tiles = B * Hkv
+        m = 1
+    else:
+        raise ValueError(mode)
+    gaps = torch.empty((tiles, nb), dtype=torch.float32, device=q.device)
+    opts = Opts(mode=m, num_splits=num_splits, gaps_out=gaps.data_ptr())
+    mk, c = _attn("blasst_calibrate", q, k, None, scale=scale, lam=lam, causal=causal, o=None, lse=None,
+                  want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=tiles,
+                  n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=d)
+    return gaps, mk, c
+
+
+def calibrate_fit(L, lam, sparsity):
+    """Host least squares of ln(lambda*L) = ln(alpha) + beta*s.  Returns (alpha, beta)."""
+    import numpy as np
+
+    L = np.ascontiguousarray(L, dtype=np.float64)
+    lam = np.ascontiguousarray(lam, dtype=np.float64)
+    s = np.ascontiguousarray(sparsity, dtype=np.float64)
+    a = ctypes.c_double()
+    b = ctypes.c_double()
+    _check(lib().blasst_calibrate_fit(L.ctypes.data, lam.ctypes.data, s.ctypes.data, len(s), ctypes.byref(a),
+                                      ctypes.byref(b)), "blasst_calibrate_fit")
+    return a.value, b.value
+
+
+def calibrate_threshold(gaps_host, target):
+    """lambda for a target sparsity from host gaps (numpy float32).  Returns (lambda, achieved)."""
+    import numpy as np
+
+    g = np.ascontiguousarray(gaps_host, dtype=np.float32).ravel()
+    lam = ctypes.c_double()
+    ach = ctypes.c_double()
+    _check(lib().blasst_calibrate_threshold(g.ctypes.data, g.size, float(target), ctypes.byref(lam),
+                                            ctypes.byref(ach)), "blasst_calibrate_threshold")
+    return lam.value, ach.value
+
+
+def visited_pairs(B, Hq, Hkv, Lq, Lk, causal, is_decode) -> int:
+    opts = Opts()
+    return int(lib().blasst_visited_pairs(B, Hq, Hkv, Lq, Lk, int(bool(causal)), int(bool(is_decode)),
+                                          ctypes.byref(opts)))
+
+
+def decode_workspace_bytes(B, Hq, Lq, dv=128, num_splits=16) -> int:
+    return int(lib().blasst_decode_workspace_bytes(B, Hq, Lq, dv, num_splits))

@@ -1,0 +1,398 @@
+// blasst_api.cu -- the extern "C" boundary of libblasst.so: argument checks,
+// TMA descriptors, workspace, and the kernel launches.  No compute here.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/blasst.h"
+#include "internal.h"
+
+using namespace blasst;
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+blasst_status cuda_fail(cudaError_t e, const char *where) {
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: %s", where, cudaGetErrorString(e));
+    return BLASST_ERR_CUDA;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 3-D bf16 view [outer, rows, cols] with row stride `row_stride` elements and
+// outer stride rows*row_stride; box of box_cols x box_rows x 1, 128B swizzle.
+blasst_status make_tmap(CUtensorMap *m, const void *base, long long cols, long long rows, long long outer,
+                        long long row_stride, int box_cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return BLASST_ERR_CUDA;
+    }
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+    cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)rows * row_stride * 2};
+    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return BLASST_ERR_CUDA;
+    }
+    return BLASST_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Copy of the caller's options with fields past struct_size zeroed.
+blasst_opts read_opts(const blasst_opts *o) {
+    blasst_opts r;
+    std::memset(&r, 0, sizeof r);
+    if (o) {
+        size_t n = std::min(o->struct_size, sizeof r);
+        if (n > 0) std::memcpy(&r, o, n);
+    }
+    r.struct_size = sizeof r;
+    return r;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Common {
+    int dv;
+    long long krs, vrs;
+};
+
+blasst_status check_common(const void *q, const void *k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                           float lambda, int causal, const blasst_opts &o, Common *c) {
+    if (!q || !k) return BLASST_ERR_INVALID;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return BLASST_ERR_INVALID;
+    if (Hq % Hkv != 0) return BLASST_ERR_INVALID;
+    if (!(std::isfinite(scale) && scale > 0.f)) return BLASST_ERR_INVALID;
+    if (!(std::isfinite(lambda) && lambda >= 0.f && lambda < 1.f)) return BLASST_ERR_INVALID;
+    if (causal && Lq > Lk) return BLASST_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(k, 16)) return BLASST_ERR_INVALID;
+    c->dv = o.dv ? o.dv : d;
+    c->krs = o.k_row_stride ? o.k_row_stride : d;
+    c->vrs = o.v_row_stride ? o.v_row_stride : c->dv;
+    if (c->dv <= 0 || c->krs < d || c->vrs < c->dv || c->krs % 8 || c->vrs % 8) return BLASST_ERR_INVALID;
+    if (o.workspace && !aligned(o.workspace, 256)) return BLASST_ERR_INVALID;
+    return BLASST_OK;
+}
+
+float log2_threshold(float lambda) {
+    return lambda > 0.f ? (float)(std::log((double)lambda) / std::log(2.0)) : -INFINITY;
+}
+
+const double kLog2e = 1.4426950408889634;
+
+// ------------------------------------------------------------------- decode
+blasst_status run_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                         int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
+                         unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib) {
+    blasst_opts op = read_opts(opts_in);
+    Common c;
+    blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, op, &c);
+    if (st != BLASST_OK) return st;
+    if (!calib) {
+        if (!v || !o || !lse) return BLASST_ERR_INVALID;
+        if (!aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4)) return BLASST_ERR_INVALID;
+    } else if (!op.gaps_out) {
+        return BLASST_ERR_INVALID;
+    }
+    if (op.block_n != 0 && op.block_n != kDecodeBlockN) return BLASST_ERR_UNSUPPORTED;
+    if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
+    const int G = Hq / Hkv;
+    const long long R = (long long)G * Lq;
+    if (R > 16) return BLASST_ERR_UNSUPPORTED;
+    const int S = op.num_splits ? op.num_splits : 16;
+    if (S < 1 || S > 65535) return BLASST_ERR_INVALID;
+    if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;
+    const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
+    const int per_split = (nb + S - 1) / S;
+    if (per_split > kMaxBlocksPerSplit) return BLASST_ERR_UNSUPPORTED;
+
+    cudaStream_t sm = reinterpret_cast<cudaStream_t>(stream);
+    const int words = (nb + 31) / 32;
+    const size_t rows = (size_t)B * Hq * Lq;
+    const size_t need = blasst_decode_workspace_bytes(B, Hq, Lq, c.dv, S);
+
+    void *ws = op.workspace;
+    if (!calib && ws && op.workspace_bytes < need) return BLASST_ERR_WORKSPACE;
+
+    CUtensorMap tk, tv;
+    st = make_tmap(&tk, k, d, Lk, (long long)B * Hkv, c.krs, 64, 64);
+    if (st != BLASST_OK) return st;
+    if (!calib) {
+        st = make_tmap(&tv, v, c.dv, Lk, (long long)B * Hkv, c.vrs, 64, 64);
+        if (st != BLASST_OK) return st;
+    } else {
+        tv = tk;
+    }
+
+    bool own_ws = false;
+    if (!calib) {
+        if (!ws) {
+            cudaError_t e = cudaMallocAsync(&ws, need, sm);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+            own_ws = true;
+        }
+    }
+    cudaError_t e;
+    if (skip_mask) {
+        e = cudaMemsetAsync(skip_mask, 0, (size_t)B * Hkv * words * sizeof(uint32_t), sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_mask)");
+    }
+    if (skip_count) {
+        e = cudaMemsetAsync(skip_count, 0, sizeof(unsigned long long), sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_count)");
+    }
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    p.q = static_cast<const uint16_t *>(q);
+    p.part_o = calib ? nullptr : static_cast<float *>(ws);
+    p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));
+    p.skip_mask = skip_mask;
+    p.skip_count = skip_count;
+    p.gaps = op.gaps_out;
+    p.status = op.status_word;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.G = G; p.R = (int)R;
+    p.nb = nb; p.num_splits = S; p.per_split = per_split; p.words = words;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = (float)(scale * kLog2e);
+    p.thr_log2 = log2_threshold(lambda);
+    e = launch_decode(p, tk, tv, calib, R <= 8 ? 1 : 2, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "decode split kernel");
+    if (!calib) {
+        CombineParams cp;
+        cp.part_o = p.part_o;
+        cp.part_lse = p.part_lse;
+        cp.o = static_cast<uint16_t *>(o);
+        cp.lse = lse;
+        cp.rows = (int)rows;
+        cp.num_splits = S;
+        cp.dv = c.dv;
+        e = launch_combine(cp, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel");
+    }
+    if (own_ws) {
+        e = cudaFreeAsync(ws, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    }
+    return BLASST_OK;
+}
+
+// ------------------------------------------------------------------ prefill
+blasst_status run_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                          int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
+                          unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib) {
+    blasst_opts op = read_opts(opts_in);
+    Common c;
+    blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, op, &c);
+    if (st != BLASST_OK) return st;
+    if (!calib) {
+        if (!v || !o || !lse) return BLASST_ERR_INVALID;
+        if (!aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4)) return BLASST_ERR_INVALID;
+    } else if (!op.gaps_out) {
+        return BLASST_ERR_INVALID;
+    }
+    if (op.block_n != 0 && op.block_n != kPrefillBlockN) return BLASST_ERR_UNSUPPORTED;
+    if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
+    if (B > 65535) return BLASST_ERR_UNSUPPORTED;
+    const int nq = (Lq + kPrefillBlockM - 1) / kPrefillBlockM;
+    const int nb = (Lk + kPrefillBlockN - 1) / kPrefillBlockN;
+    const int words = (nb + 31) / 32;
+    cudaStream_t sm = reinterpret_cast<cudaStream_t>(stream);
+
+    CUtensorMap tq, tk, tv;
+    st = make_tmap(&tq, q, d, Lq, (long long)B * Hq, d, 64, kPrefillBlockM);
+    if (st != BLASST_OK) return st;
+    st = make_tmap(&tk, k, d, Lk, (long long)B * Hkv, c.krs, 64, kPrefillBlockN);
+    if (st != BLASST_OK) return st;
+    if (!calib) {
+        st = make_tmap(&tv, v, c.dv, Lk, (long long)B * Hkv, c.vrs, 64, kPrefillBlockN);
+        if (st != BLASST_OK) return st;
+    } else {
+        tv = tk;
+    }
+    cudaError_t e;
+    if (skip_count) {
+        e = cudaMemsetAsync(skip_count, 0, sizeof(unsigned long long), sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_count)");
+    }
+    PrefillParams p;
+    std::memset(&p, 0, sizeof p);
+    p.o = static_cast<uint16_t *>(o);
+    p.lse = lse;
+    p.skip_mask = skip_mask;
+    p.skip_count = skip_count;
+    p.gaps = op.gaps_out;
+    p.status = op.status_word;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.G = Hq / Hkv;
+    p.n_qtiles = nq; p.nb = nb; p.words = words;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = (float)(scale * kLog2e);
+    p.thr_log2 = log2_threshold(lambda);
+    e = launch_prefill(p, tq, tk, tv, calib, sm);
+    if (e == cudaErrorNotSupported) return BLASST_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return cuda_fail(e, "prefill kernel");
+    return BLASST_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+blasst_status blasst_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                             int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
+                             unsigned long long *skip_count, void *stream, const blasst_opts *opts) {
+    return run_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
+                       opts, false);
+}
+
+blasst_status blasst_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                            int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
+                            unsigned long long *skip_count, void *stream, const blasst_opts *opts) {
+    return run_decode(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
+                      opts, false);
+}
+
+blasst_status blasst_calibrate(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                               int Hkv, int Lq, int Lk, int d, float scale, float lambda, int causal,
+                               uint32_t *skip_mask, unsigned long long *skip_count, void *stream,
+                               const blasst_opts *opts) {
+    (void)v;
+    (void)o;
+    (void)lse;
+    blasst_opts op = read_opts(opts);
+    if (op.mode == 1)
+        return run_decode(q, k, nullptr, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask,
+                          skip_count, stream, opts, true);
+    if (op.mode != 0) return BLASST_ERR_INVALID;
+    return run_prefill(q, k, nullptr, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask,
+                       skip_count, stream, opts, true);
+}
+
+blasst_status blasst_calibrate_fit(const double *L, const double *lambda, const double *sparsity, int n,
+                                   double *alpha, double *beta) {
+    if (!L || !lambda || !sparsity || !alpha || !beta || n < 2) return BLASST_ERR_INVALID;
+    double sx = 0, sy = 0, sxx = 0, sxy = 0;
+    for (int i = 0; i < n; i++) {
+        if (!(L[i] > 0) || !(lambda[i] > 0) || !std::isfinite(sparsity[i])) return BLASST_ERR_INVALID;
+        const double x = sparsity[i], y = std::log(lambda[i] * L[i]);
+        sx += x;
+        sy += y;
+        sxx += x * x;
+        sxy += x * y;
+    }
+    const double den = n * sxx - sx * sx;
+    if (den == 0.0) return BLASST_ERR_INVALID;
+    *beta = (n * sxy - sx * sy) / den;
+    *alpha = std::exp((sy - *beta * sx) / n);
+    return BLASST_OK;
+}
+
+blasst_status blasst_calibrate_threshold(const float *gaps, long long n, double target, double *lambda_out,
+                                         double *achieved_out) {
+    if (!gaps || n < 0 || !lambda_out || !(target >= 0.0 && target <= 1.0)) return BLASST_ERR_INVALID;
+    long long n_vis = 0;
+    std::vector<double> cand;
+    for (long long i = 0; i < n; i++) {
+        const float g = gaps[i];
+        if (std::isnan(g)) continue;
+        n_vis++;
+        if (std::isfinite(g) && g < 0.f) cand.push_back((double)g);
+    }
+    std::sort(cand.begin(), cand.end());
+    long long want = n_vis ? (long long)std::llround(target * (double)n_vis) : 0;
+    want = std::max(0LL, std::min<long long>(want, (long long)cand.size()));
+    double lam = 0.0;
+    long long got = 0;
+    if (want > 0) {
+        const double lo = cand[want - 1];
+        const double hi = want < (long long)cand.size() ? cand[want] : 0.0;
+        double ln_lam = hi > lo ? 0.5 * (lo + hi) : std::nextafter(lo, INFINITY);
+        lam = std::min(std::exp(ln_lam), std::nextafter(1.0, 0.0));
+        // what the device decides: gap (log2 units, fp32) < log2(lambda) (fp32)
+        const float thr = log2_threshold((float)lam);
+        for (double g : cand)
+            if ((float)((float)g * (float)kLog2e) < thr) got++;
+    }
+    *lambda_out = lam;
+    if (achieved_out) *achieved_out = n_vis ? (double)got / (double)n_vis : 0.0;
+    return BLASST_OK;
+}
+
+size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_splits) {
+    if (B <= 0 || Hq <= 0 || Lq <= 0 || dv < 0 || num_splits < 0) return 0;
+    const size_t S = num_splits ? num_splits : 16;
+    const size_t rows = (size_t)B * Hq * Lq;
+    const size_t dvv = dv ? dv : 128;
+    return round_up(rows * S * dvv * 4, 256) + round_up(rows * S * 4, 256);
+}
+
+long long blasst_visited_pairs(int B, int Hq, int Hkv, int Lq, int Lk, int causal, int is_decode,
+                               const blasst_opts *opts) {
+    blasst_opts op = read_opts(opts);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || Hq % Hkv) return -1;
+    if (causal && Lq > Lk) return -1;
+    if (is_decode) {
+        const int bn = op.block_n ? op.block_n : kDecodeBlockN;
+        const long long nb = (Lk + bn - 1) / bn;
+        // every key block is seen by the last query of the tile
+        return (long long)B * Hkv * nb;
+    }
+    const int bn = op.block_n ? op.block_n : kPrefillBlockN;
+    const long long nb = (Lk + bn - 1) / bn;
+    const int nq = (Lq + kPrefillBlockM - 1) / kPrefillBlockM;
+    long long per_head = 0;
+    for (int t = 0; t < nq; t++) {
+        if (!causal) {
+            per_head += nb;
+        } else {
+            const long long last_row = std::min<long long>(Lq, (long long)(t + 1) * kPrefillBlockM) - 1;
+            const long long last_key = last_row + (Lk - Lq);
+            per_head += std::min<long long>(nb, last_key / bn + 1);
+        }
+    }
+    return per_head * B * Hq;
+}
+
+const char *blasst_status_string(blasst_status s) {
+    switch (s) {
+        case BLASST_OK: return "ok";
+        case BLASST_ERR_INVALID: return "invalid argument";
+        case BLASST_ERR_UNSUPPORTED: return "unsupported configuration";
+        case BLASST_ERR_WORKSPACE: return "workspace too small";
+        case BLASST_ERR_CUDA: return "CUDA error";
+        case BLASST_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *blasst_last_error(void) { return g_last_error; }
+
+}  // extern "C"

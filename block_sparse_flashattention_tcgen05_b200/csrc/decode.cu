@@ -1,0 +1,472 @@
+// decode.cu -- split-KV decode with softmax-threshold block skipping (BLASST),
+// and the lse combine of the splits.
+//
+// One CTA per (split, KV head, sequence).  The tile is the G query heads x Lq
+// queries that share the KV head (G*Lq <= 8*NT rows).  KV blocks are 64 keys.
+//
+// Warp roles (192 threads):
+//   warps 0-3  consumers: each owns 16 keys of every block.  S^T = K_j q^T on
+//              the tensor cores (mma.sync m16n8k16, keys on M, query rows on
+//              N), block row maxima exchanged through shared memory, the
+//              tile-wide skip decision, then for kept blocks exp2 and
+//              O^T += V_j^T P^T (P re-laid out in registers with movmatrix).
+//   warp 4     K producer: TMA loads of K blocks into a ring, as far ahead as
+//              the ring allows; K is read for every block.
+//   warp 5     V producer: waits for each block's published decision and
+//              issues the TMA load of V_j only for kept blocks.  The decision
+//              is taken before any V traffic for the block (xllm-io paper
+//              review, section 3 "decode kernel optimisation": V_j of pruned
+//              blocks is never loaded; gist.science (de) section 3: batched,
+//              conditional V loads after the key blocks).
+//
+// The running max per row restarts in every split; the first visited block
+// of a split is always kept.  Scores are handled in log2 units:
+// s2 = (q.k) * scale * log2(e), compared with log2(lambda).
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace blasst {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 64;
+constexpr int kStageBytes = kDecodeBlockN * 128 * 2;  // 64 keys x 128 dims bf16
+constexpr int kBoxBytes = kStageBytes / 2;             // 64 keys x 64 dims (one 128-byte swizzle box)
+constexpr int kStatusTimeout = 1;
+
+struct DecodeSmemTail {
+    uint64_t k_full[8];
+    uint64_t k_empty[8];
+    uint64_t v_full[8];
+    uint64_t v_empty[8];
+    float red[2][kConsumerWarps][16];
+    float lred[kConsumerWarps][16];
+    float mfin[16];
+    int dec_count;
+    int abort;
+};
+
+template <int NK, int NV, bool CALIB>
+constexpr int decode_smem_bytes() {
+    return NK * kStageBytes + (CALIB ? 0 : NV * kStageBytes) + (int)sizeof(DecodeSmemTail) + kMaxBlocksPerSplit + 1024;
+}
+
+__device__ __forceinline__ void set_timeout(DecodeSmemTail *t, unsigned int *status) {
+    t->abort = 1;
+    if (status) atomicOr(status, kStatusTimeout);
+}
+
+template <int NT, int NK, int NV, bool CALIB>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *kring = smem;
+    uint8_t *vring = smem + NK * kStageBytes;
+    DecodeSmemTail *tl = reinterpret_cast<DecodeSmemTail *>(vring + (CALIB ? 0 : NV * kStageBytes));
+    volatile uint8_t *dec = reinterpret_cast<volatile uint8_t *>(tl + 1);
+
+    const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j0 = split * p.per_split;
+    const int j1 = min(p.nb, j0 + p.per_split);
+    const int nblk = max(0, j1 - j0);
+    const int bh = b * p.Hkv + hkv;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NK; i++) {
+            mbar_init(&tl->k_full[i], 1);
+            mbar_init(&tl->k_empty[i], kConsumerWarps);
+        }
+        if (!CALIB) {
+            for (int i = 0; i < NV; i++) {
+                mbar_init(&tl->v_full[i], 1);
+                mbar_init(&tl->v_empty[i], kConsumerWarps);
+            }
+        }
+        tl->dec_count = 0;
+        tl->abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ K producer
+    if (warp == kConsumerWarps) {
+        if (lane != 0) return;
+        tma_prefetch_desc(&tmap_k);
+        int issued = 0;
+        for (int jj = 0; jj < nblk; jj++) {
+            const int slot = jj % NK;
+            if (jj >= NK && !mbar_wait(&tl->k_empty[slot], ((jj / NK) & 1) ^ 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
+            uint8_t *dst = kring + slot * kStageBytes;
+            mbar_arrive_expect_tx(&tl->k_full[slot], kStageBytes);
+            tma_load_3d(dst, &tmap_k, &tl->k_full[slot], 0, (j0 + jj) * kDecodeBlockN, bh);
+            tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, (j0 + jj) * kDecodeBlockN, bh);
+            issued++;
+        }
+        if (tl->abort) {  // let copies in flight land before the CTA exits
+            for (int jj = max(0, issued - NK); jj < issued; jj++) mbar_wait(&tl->k_full[jj % NK], (jj / NK) & 1, nullptr);
+        }
+        return;
+    }
+    // ------------------------------------------------------------ V producer
+    if (warp == kConsumerWarps + 1) {
+        if (CALIB || lane != 0) return;
+        tma_prefetch_desc(&tmap_v);
+        int vk = 0;
+        for (int jj = 0; jj < nblk && !tl->abort; jj++) {
+            long long t0 = clock64();
+            while (*reinterpret_cast<volatile int *>(&tl->dec_count) <= jj) {
+                if (tl->abort || clock64() - t0 > kWaitLimitCycles) {
+                    set_timeout(tl, p.status);
+                    break;
+                }
+            }
+            if (tl->abort) break;
+            __threadfence_block();
+            if (!dec[jj]) continue;
+            const int slot = vk % NV;
+            if (vk >= NV && !mbar_wait(&tl->v_empty[slot], ((vk / NV) & 1) ^ 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
+            uint8_t *dst = vring + slot * kStageBytes;
+            mbar_arrive_expect_tx(&tl->v_full[slot], kStageBytes);
+            tma_load_3d(dst, &tmap_v, &tl->v_full[slot], 0, (j0 + jj) * kDecodeBlockN, bh);
+            tma_load_3d(dst + kBoxBytes, &tmap_v, &tl->v_full[slot], 64, (j0 + jj) * kDecodeBlockN, bh);
+            vk++;
+        }
+        if (tl->abort) {
+            for (int i = max(0, vk - NV); i < vk; i++) mbar_wait(&tl->v_full[i % NV], (i / NV) & 1, nullptr);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------- consumers
+    const int g4 = lane >> 2, t4 = lane & 3;
+    constexpr int NC = 8 * NT;  // padded tile rows (columns of S^T)
+    const int qrow0 = (b * p.Hq + hkv * p.G) * p.Lq;  // flat row index of tile row 0
+
+    // q^T as mma B fragments, for all 8 k-steps of d = 128
+    uint32_t qf[8][NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; nt++) {
+        const int n = nt * 8 + g4;
+        const uint32_t *qr = reinterpret_cast<const uint32_t *>(p.q + (size_t)(qrow0 + min(n, p.R - 1)) * 128);
+#pragma unroll
+        for (int ks = 0; ks < 8; ks++) {
+            qf[ks][nt][0] = n < p.R ? __ldg(qr + ks * 8 + t4) : 0u;
+            qf[ks][nt][1] = n < p.R ? __ldg(qr + ks * 8 + 4 + t4) : 0u;
+        }
+    }
+    // last visible key of each of my columns (col = nt*8 + 2*t4 + e)
+    int lastk[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int c = nt * 8 + 2 * t4 + e;
+            const int pos = c % p.Lq;
+            lastk[nt][e] = c >= p.R ? -1 : (p.causal ? pos + (p.Lk - p.Lq) : p.Lk - 1);
+        }
+
+    float Mall[NC];
+#pragma unroll
+    for (int c = 0; c < NC; c++) Mall[c] = -CUDART_INF_F;
+    float o_acc[CALIB ? 1 : 8][NT][4];
+    float lsum[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; nt++) {
+        lsum[nt][0] = lsum[nt][1] = 0.f;
+        if (!CALIB)
+#pragma unroll
+            for (int mt = 0; mt < 8; mt++)
+#pragma unroll
+                for (int i = 0; i < 4; i++) o_acc[mt][nt][i] = 0.f;
+    }
+
+    bool seen = false;
+    int kept_count = 0;
+    uint32_t mask_word = 0;
+    int mask_word_idx = -1;
+    unsigned long long n_skip = 0;
+    const float NEG_INF = -CUDART_INF_F;
+
+    for (int jj = 0; jj < nblk; jj++) {
+        const int j = j0 + jj;
+        const int slot = jj % NK;
+        if (!mbar_wait(&tl->k_full[slot], (jj / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
+        const uint8_t *kb = kring + slot * kStageBytes;
+
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        {
+            const int mi = lane >> 3, ri = lane & 7;
+            const int key = warp * 16 + ri + 8 * (mi & 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++) {
+                const int chunk = ks * 2 + (mi >> 1);
+                uint32_t a[4];
+                ldsm_x4(smem_addr(kb + (chunk >> 3) * kBoxBytes + swz128(key, chunk & 7)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) mma_bf16_16816(acc[nt], a, qf[ks][nt]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl->k_empty[slot]);
+
+        // scaled, masked scores in log2 units; my keys: lo = g4, hi = g4 + 8
+        const int key_lo = j * kDecodeBlockN + warp * 16 + g4;
+        float s[NT][4];
+        float cmax[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                s[nt][e] = key_lo <= lastk[nt][e] && key_lo < p.Lk ? acc[nt][e] * p.scale_log2 : NEG_INF;
+                s[nt][2 + e] = key_lo + 8 <= lastk[nt][e] && key_lo + 8 < p.Lk ? acc[nt][2 + e] * p.scale_log2 : NEG_INF;
+                float m = fmaxf(s[nt][e], s[nt][2 + e]);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                cmax[nt][e] = m;
+            }
+        }
+        if (g4 == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++) {
+                tl->red[jj & 1][warp][nt * 8 + 2 * t4] = cmax[nt][0];
+                tl->red[jj & 1][warp][nt * 8 + 2 * t4 + 1] = cmax[nt][1];
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+
+        // block row maxima of the whole tile, running max after the block, gap
+        float Mn[NC];
+        float gap = NEG_INF;
+        bool visited = false;
+#pragma unroll
+        for (int c = 0; c < NC; c++) {
+            float mt = tl->red[jj & 1][0][c];
+#pragma unroll
+            for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[jj & 1][w][c]);
+            Mn[c] = fmaxf(Mall[c], mt);
+            if (mt > NEG_INF) {
+                visited = true;
+                gap = fmaxf(gap, mt - Mn[c]);
+            }
+        }
+        const bool first = visited && !seen;
+        seen = seen || visited;
+        const bool skip = visited && !first && (gap < p.thr_log2);
+        const bool kept = visited && !skip;
+
+        if (warp == 0 && lane == 0) {
+            if (!CALIB) {
+                dec[jj] = kept ? 1 : 0;
+                __threadfence_block();
+                *reinterpret_cast<volatile int *>(&tl->dec_count) = jj + 1;
+            }
+            if (p.gaps)
+                p.gaps[(size_t)bh * p.nb + j] =
+                    !visited ? CUDART_NAN_F : (first ? CUDART_INF_F : gap * 0.69314718055994531f);
+            if (skip) {
+                n_skip++;
+                if (p.skip_mask) {
+                    if (mask_word_idx != (j >> 5)) {
+                        if (mask_word_idx >= 0 && mask_word)
+                            atomicOr(p.skip_mask + (size_t)bh * p.words + mask_word_idx, mask_word);
+                        mask_word_idx = j >> 5;
+                        mask_word = 0;
+                    }
+                    mask_word |= 1u << (j & 31);
+                }
+            }
+        }
+        if (CALIB) {
+            if (kept) {
+#pragma unroll
+                for (int c = 0; c < NC; c++) Mall[c] = Mn[c];
+            }
+            continue;
+        }
+        if (!kept) continue;
+
+        // rescale by the growth of the running max, then P = 2^(s - M)
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                const int c = nt * 8 + 2 * t4 + e;
+                float mold = NEG_INF, mnew = NEG_INF;
+#pragma unroll
+                for (int cc = 0; cc < NC; cc++)
+                    if (cc == c) {
+                        mold = Mall[cc];
+                        mnew = Mn[cc];
+                    }
+                const float alpha = (mnew == NEG_INF) ? 1.f : ex2(mold - mnew);
+                lsum[nt][e] *= alpha;
+#pragma unroll
+                for (int mt = 0; mt < 8; mt++) {
+                    o_acc[mt][nt][e] *= alpha;
+                    o_acc[mt][nt][2 + e] *= alpha;
+                }
+                pv[e] = s[nt][e] == NEG_INF ? 0.f : ex2(s[nt][e] - mnew);
+                pv[2 + e] = s[nt][2 + e] == NEG_INF ? 0.f : ex2(s[nt][2 + e] - mnew);
+                lsum[nt][e] += pv[e] + pv[2 + e];
+            }
+            pb[nt][0] = movmatrix_t(pack_bf16x2(pv[0], pv[1]));
+            pb[nt][1] = movmatrix_t(pack_bf16x2(pv[2], pv[3]));
+        }
+#pragma unroll
+        for (int c = 0; c < NC; c++) Mall[c] = Mn[c];
+
+        const int vslot = kept_count % NV;
+        if (!mbar_wait(&tl->v_full[vslot], (kept_count / NV) & 1, &tl->abort)) set_timeout(tl, p.status);
+        const uint8_t *vb = vring + vslot * kStageBytes;
+        {
+            const int mi = lane >> 3, ri = lane & 7;
+            const int key = warp * 16 + ri + 8 * (mi >> 1);
+#pragma unroll
+            for (int mt = 0; mt < 8; mt++) {
+                const int chunk = mt * 2 + (mi & 1);
+                uint32_t a[4];
+                ldsm_x4_t(smem_addr(vb + (chunk >> 3) * kBoxBytes + swz128(key, chunk & 7)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) mma_bf16_16816(o_acc[mt][nt], a, pb[nt]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl->v_empty[vslot]);
+        kept_count++;
+    }
+
+    if (warp == 0 && lane == 0) {
+        if (p.skip_mask && mask_word_idx >= 0 && mask_word)
+            atomicOr(p.skip_mask + (size_t)bh * p.words + mask_word_idx, mask_word);
+        if (p.skip_count && n_skip) atomicAdd(p.skip_count, n_skip);
+    }
+    if (CALIB) return;
+
+    // ------------------------------------------------ reduce over the 4 warps
+    // partial O^T of each warp -> shared memory (the K ring is idle now)
+    float *obuf = reinterpret_cast<float *>(kring);  // [warp][dv 128][NC]
+#pragma unroll
+    for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            float l = lsum[nt][e];
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            if (g4 == 0) tl->lred[warp][nt * 8 + 2 * t4 + e] = l;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; mt++) {
+            const int dv0 = mt * 16 + g4;
+            const int c0 = nt * 8 + 2 * t4;
+            obuf[(warp * 128 + dv0) * NC + c0] = o_acc[mt][nt][0];
+            obuf[(warp * 128 + dv0) * NC + c0 + 1] = o_acc[mt][nt][1];
+            obuf[(warp * 128 + dv0 + 8) * NC + c0] = o_acc[mt][nt][2];
+            obuf[(warp * 128 + dv0 + 8) * NC + c0 + 1] = o_acc[mt][nt][3];
+        }
+    }
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int c = 0; c < NC; c++) tl->mfin[c] = Mall[c];
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+
+    const int x = threadIdx.x;  // dv index 0..127
+    const int S = p.num_splits;
+    for (int c = 0; c < p.R; c++) {
+        float l = 0.f, o = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; w++) {
+            l += tl->lred[w][c];
+            o += obuf[(w * 128 + x) * NC + c];
+        }
+        const size_t row = (size_t)(qrow0 + c) * S + split;
+        p.part_o[row * 128 + x] = l > 0.f ? o / l : 0.f;
+        if (x == 0) p.part_lse[row] = l > 0.f ? (tl->mfin[c] + __log2f(l)) * 0.69314718055994531f : NEG_INF;
+    }
+}
+
+// One warp per output row: lse = ln sum_s exp(lse_s); O = sum_s exp(lse_s - lse) O_s.
+__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= p.rows) return;
+    const int S = p.num_splits;
+    const float LOG2E = 1.4426950408889634f;
+    float mx = -CUDART_INF_F;
+    for (int s = lane; s < S; s += 32) mx = fmaxf(mx, p.part_lse[(size_t)row * S + s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+    if (mx > -CUDART_INF_F)
+        for (int s = lane; s < S; s += 32) sum += ex2((p.part_lse[(size_t)row * S + s] - mx) * LOG2E);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float L = mx > -CUDART_INF_F ? mx + __logf(sum) : -CUDART_INF_F;
+    for (int x0 = lane * 4; x0 < p.dv; x0 += 128) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (L > -CUDART_INF_F) {
+            for (int s = 0; s < S; s++) {
+                const float ls = p.part_lse[(size_t)row * S + s];
+                if (ls == -CUDART_INF_F) continue;
+                const float w = ex2((ls - L) * LOG2E);
+                const float4 v = *reinterpret_cast<const float4 *>(p.part_o + ((size_t)row * S + s) * p.dv + x0);
+                acc[0] += w * v.x;
+                acc[1] += w * v.y;
+                acc[2] += w * v.z;
+                acc[3] += w * v.w;
+            }
+        }
+        uint2 packed;
+        packed.x = pack_bf16x2(acc[0], acc[1]);
+        packed.y = pack_bf16x2(acc[2], acc[3]);
+        *reinterpret_cast<uint2 *>(p.o + (size_t)row * p.dv + x0) = packed;
+    }
+    if (lane == 0) p.lse[row] = L;
+}
+
+template <int NT, bool CALIB>
+cudaError_t launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st) {
+    constexpr int NK = 4, NV = 2;
+    constexpr int smem = decode_smem_bytes<NK, NV, CALIB>();
+    auto kern = decode_split_kernel<NT, NK, NV, CALIB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.num_splits, p.Hkv, p.B);
+    kern<<<grid, kThreads, smem, st>>>(p, tk, tv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, bool calib, int nt,
+                          cudaStream_t st) {
+    if (calib) return nt == 1 ? launch_decode_t<1, true>(p, tk, tv, st) : launch_decode_t<2, true>(p, tk, tv, st);
+    return nt == 1 ? launch_decode_t<1, false>(p, tk, tv, st) : launch_decode_t<2, false>(p, tk, tv, st);
+}
+
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t st) {
+    if (p.rows == 0) return cudaSuccess;
+    combine_kernel<<<(p.rows + 3) / 4, 128, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace blasst

@@ -1,0 +1,62 @@
+// internal.h -- parameters shared between the C-ABI host layer and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace blasst {
+
+constexpr int kDecodeBlockN = 64;
+constexpr int kPrefillBlockM = 128;
+constexpr int kPrefillBlockN = 128;
+constexpr int kMaxBlocksPerSplit = 8192;
+
+// One decode (or decode-shaped calibration) call.
+struct DecodeParams {
+    const uint16_t *q;              // [B, Hq, Lq, d] bf16
+    float *part_o;                  // [B*Hq*Lq, S, dv] fp32 split outputs (normalised)
+    float *part_lse;                // [B*Hq*Lq, S] fp32 split lse (natural log)
+    uint32_t *skip_mask;            // [B, Hkv, 1, W] or null
+    unsigned long long *skip_count; // or null
+    float *gaps;                    // [B*Hkv, nb] or null
+    unsigned int *status;           // or null
+    int B, Hq, Hkv, Lq, Lk, G, R;   // R = G * Lq rows per tile
+    int nb, num_splits, per_split, words;
+    int causal;
+    float scale_log2;               // scale * log2(e)
+    float thr_log2;                 // log2(lambda), -inf for lambda = 0
+};
+
+struct CombineParams {
+    const float *part_o;
+    const float *part_lse;
+    uint16_t *o;      // [B, Hq, Lq, dv] bf16
+    float *lse;       // [B, Hq, Lq]
+    int rows;         // B * Hq * Lq
+    int num_splits;
+    int dv;
+};
+
+// One prefill (or prefill-shaped calibration) call.
+struct PrefillParams {
+    uint16_t *o;                    // [B, Hq, Lq, 128] bf16
+    float *lse;                     // [B, Hq, Lq]
+    uint32_t *skip_mask;            // [B, Hq, n_qtiles, W] or null
+    unsigned long long *skip_count; // or null
+    float *gaps;                    // [B*Hq*n_qtiles, nb] or null
+    unsigned int *status;           // or null
+    int B, Hq, Hkv, Lq, Lk, G;
+    int n_qtiles, nb, words;
+    int causal;
+    float scale_log2;
+    float thr_log2;
+};
+
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
+                          int nt, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                           const CUtensorMap &tmap_v, bool calib, cudaStream_t stream);
+
+}  // namespace blasst

@@ -1,0 +1,176 @@
+/*
+ * blasst.h -- C ABI of libblasst.so: BLASST blocked attention with
+ * softmax-threshold block skipping on NVIDIA B200 (sm_100a).
+ *
+ * The method (BLASST: "Dynamic BLocked Attention Sparsity via Softmax
+ * Thresholding", arXiv:2512.12087):
+ *   attention = softmax(Q K^T * scale) V  (xllm-io paper review, section 3,
+ *   "core formulas"), computed FlashAttention-style over KV blocks in order
+ *   with a running row max m.  A KV block j is skipped for a query tile when
+ *   every row r of the tile that sees a key of the block satisfies
+ *       m~_r(j) - max(m_r, m~_r(j)) < ln(lambda)
+ *   where m~_r(j) is the row max of the block's scaled scores (same section,
+ *   skip condition; gist.science (de) summary, section 2 "Kernidee").  A
+ *   skipped block adds nothing to the row sum l or to O; its exp, its V load
+ *   (decode) and its P.V product are not done (gist.science (de), section 2;
+ *   fugumt abstract).  The first visited block of a tile is never skipped
+ *   (nervesearch commentary, six-block figure).  lambda = 0 means dense.
+ *
+ * Conventions common to every entry point
+ *   - Tensors are row-major and head-major: q [B, Hq, Lq, d], k [B, Hkv, Lk,
+ *     *], v [B, Hkv, Lk, *], o [B, Hq, Lq, dv] in bf16 (raw 16-bit words),
+ *     lse [B, Hq, Lq] fp32 natural-log logsumexp of the kept scores.  k and v
+ *     rows hold k_row_stride / v_row_stride elements (default d / dv), so an
+ *     MLA latent cache can pass the same buffer as k and v with dv < d.
+ *   - Every pointer argument is a DEVICE pointer (except in the host-only
+ *     functions marked so).  q, k, v, o must be 16-byte aligned; row strides
+ *     must be multiples of 8 elements.  The caller owns every buffer; the
+ *     library keeps no per-call state (TMA descriptors are built on the host
+ *     for each call), and calls on different streams may run concurrently.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns; results are ready when the stream
+ *     is synchronised.
+ *   - Causal masking is aligned bottom-right: query i may see keys
+ *     0 .. i + (Lk - Lq).  causal requires Lq <= Lk.
+ *   - lambda must be finite with 0 <= lambda < 1; scale must be > 0.
+ *   - skip_mask (nullable) receives one bit per (query tile, KV block), 1 =
+ *     skipped, as rows of W = ceil(n_blocks / 32) uint32 words: bit (j % 32)
+ *     of word (j / 32) is block j.  Prefill: rows [B, Hq, ceil(Lq / 128)],
+ *     128 queries per tile, blocks of 128 keys.  Decode: rows [B, Hkv, 1], the
+ *     tile being all G = Hq/Hkv query heads x Lq queries of one KV head,
+ *     blocks of 64 keys.  The library writes every word of the mask (blocks a
+ *     tile never visits read 0).
+ *   - skip_count (nullable) is one uint64 on the device: the library sets it
+ *     to the number of skipped (tile, block) pairs of the call.  The
+ *     denominator, visited pairs, comes from blasst_visited_pairs().
+ *   - Errors: invalid arguments return BLASST_ERR_INVALID / _UNSUPPORTED /
+ *     _WORKSPACE before anything is enqueued; a failed CUDA call returns
+ *     BLASST_ERR_CUDA (text via blasst_last_error()).  Device-side bounded
+ *     waits that time out write a nonzero code into opts->status_word (when
+ *     given) and make the kernel return early; the host sees it after
+ *     synchronising.  No C++ exception crosses this interface.
+ */
+#ifndef BLASST_H
+#define BLASST_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BLASST_API __attribute__((visibility("default")))
+#else
+#define BLASST_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BLASST_OK = 0,
+    BLASST_ERR_INVALID = 1,     /* bad pointer, shape, scale or lambda */
+    BLASST_ERR_UNSUPPORTED = 2, /* valid in principle, not built (e.g. head dim) */
+    BLASST_ERR_WORKSPACE = 3,   /* caller's workspace too small */
+    BLASST_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    BLASST_ERR_TIMEOUT = 5      /* device status word: a bounded wait expired */
+} blasst_status;
+
+/* Optional arguments; pass NULL for all defaults.  struct_size must be
+ * sizeof(blasst_opts) as compiled by the caller (ABI versioning): fields past
+ * struct_size are treated as zero. */
+typedef struct blasst_opts {
+    size_t struct_size;
+    int dv;                    /* value head dim; 0 -> d.  MLA: d = 576, dv = 512 */
+    int block_n;               /* 0, or the fixed block size (128 prefill, 64 decode) */
+    int num_splits;            /* decode: KV chunks per sequence; 0 -> 16 */
+    int mode;                  /* blasst_calibrate only: 0 = prefill tiling, 1 = decode tiling */
+    long long k_row_stride;    /* elements between consecutive keys; 0 -> d */
+    long long v_row_stride;    /* elements between consecutive values; 0 -> dv */
+    void *workspace;           /* decode partials; NULL -> stream-ordered cudaMallocAsync */
+    size_t workspace_bytes;
+    float *gaps_out;           /* device, per (tile, block) pair: max over rows of
+                                  m~ - max(m, m~) in natural-log units; +inf on a
+                                  tile's (split's) first block, NaN if not visited */
+    unsigned int *status_word; /* device word the caller zeroes; the library ORs in
+                                  a nonzero code when a bounded wait expires */
+} blasst_opts;
+
+/*
+ * Prefill: Lq queries attend to Lk keys per sequence, query tiles of 128
+ * rows of one query head, KV blocks of 128 keys, kv head = hq / (Hq / Hkv).
+ * d = dv = 128 only.  QK^T is computed for every visited block; the skip
+ * decision then omits exp and the P.V tensor-core product of skipped blocks
+ * (xllm-io paper review, section 3 "prefill kernel optimisation").
+ */
+BLASST_API blasst_status blasst_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                             int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, float lambda,
+                             int causal, uint32_t *skip_mask, unsigned long long *skip_count,
+                             void *stream, const blasst_opts *opts);
+
+/*
+ * Decode: the G = Hq/Hkv query heads x Lq queries of one KV head form the
+ * tile (G * Lq <= 16), KV blocks of 64 keys, split-KV over num_splits
+ * contiguous chunks of ceil(n_blocks / num_splits) blocks.  Each split is an
+ * independent online-softmax pass (running max restarts, its first block is
+ * kept); the skip decision for a block is taken after its K block is read and
+ * before any load of its V block, V is loaded only for kept blocks (xllm-io
+ * paper review, section 3 "decode kernel optimisation"), then a combine step
+ * merges the splits exactly on lse.  d = dv = 128 (GQA/MQA).
+ * Workspace: blasst_decode_workspace_bytes() bytes, 256-byte aligned.
+ */
+BLASST_API blasst_status blasst_decode(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, float lambda,
+                            int causal, uint32_t *skip_mask, unsigned long long *skip_count,
+                            void *stream, const blasst_opts *opts);
+
+/*
+ * Calibration pass: the decision part of prefill (opts->mode = 0) or decode
+ * (mode = 1) only -- QK^T, block row maxima, running max, gaps -- without
+ * exp, P.V or V traffic.  v, o and lse may be NULL and are not touched.
+ * Writes opts->gaps_out (required) and, for the given lambda, skip_mask and
+ * skip_count exactly as the matching attention call would.  One pass serves
+ * every lambda: a skipped block never raises the running max, so a pair is
+ * skipped at lambda iff its gap < ln(lambda) (xllm-io paper review, section 3,
+ * "calibration module": one forward pass).
+ */
+BLASST_API blasst_status blasst_calibrate(const void *q, const void *k, const void *v, void *o, float *lse,
+                               int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, float lambda,
+                               int causal, uint32_t *skip_mask, unsigned long long *skip_count,
+                               void *stream, const blasst_opts *opts);
+
+/*
+ * HOST-ONLY.  Least-squares fit of ln(lambda_i * L_i) = ln(alpha) + beta * s_i
+ * over n >= 2 points: the calibration model lambda * L = alpha * exp(beta * s)
+ * (xllm-io paper review, section 3, "calibration model").  Host arrays.
+ */
+BLASST_API blasst_status blasst_calibrate_fit(const double *L, const double *lambda, const double *sparsity, int n,
+                                   double *alpha, double *beta);
+
+/*
+ * HOST-ONLY.  From n gaps of one calibration pass (host copy of gaps_out),
+ * the lambda whose sparsity (skipped / visited pairs) is closest to
+ * target_sparsity, and the sparsity it reaches.  NaN entries are not visited,
+ * +inf entries are first blocks (visited, never skipped).
+ */
+BLASST_API blasst_status blasst_calibrate_threshold(const float *gaps, long long n, double target_sparsity,
+                                         double *lambda_out, double *achieved_out);
+
+/* Bytes of decode workspace for these sizes (num_splits 0 -> 16, dv 0 -> 128). */
+BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_splits);
+
+/* Number of visited (tile, block) pairs: the sparsity denominator.
+ * is_decode selects the decode tiling; -1 on invalid sizes. */
+BLASST_API long long blasst_visited_pairs(int B, int Hq, int Hkv, int Lq, int Lk, int causal, int is_decode,
+                               const blasst_opts *opts);
+
+/* Static text for a status code. */
+BLASST_API const char *blasst_status_string(blasst_status s);
+
+/* Text of the last CUDA failure seen by this thread ("" if none). */
+BLASST_API const char *blasst_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLASST_H */

@@ -1,0 +1,166 @@
+"""The C-ABI library: it loads, exports what include/blasst.h declares, and its
+host-only logic (argument checks, calibration fit and threshold, visited-pair
+counts, workspace size) behaves as specified.  No GPU needed: every call here
+returns before any CUDA work."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import planted_prefill, random_normal
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bl():
+    from block_sparse_flashattention_tcgen05_b200 import build
+
+    build.build()
+    import block_sparse_flashattention_tcgen05_b200 as m
+
+    m.lib()
+    return m
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "blasst.h")) as f:
+        text = f.read()
+    return re.findall(r"BLASST_API\s+[\w\s\*]+?\b(blasst_\w+)\s*\(", text)
+
+
+def test_exports_every_declared_symbol(bl):
+    names = declared_symbols()
+    assert len(names) >= 9
+    L = bl.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+FAKE = 0x10000  # an aligned non-null address; never dereferenced on these paths
+
+
+def _call(bl, fn, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=4, Hkv=1, Lq=1, Lk=256, d=128, scale=0.088,
+                lam=0.0, causal=0, mask=None, count=None, stream=None, opts=None)
+    args.update(over)
+    opts = args["opts"] or bl.Opts()
+    f = getattr(bl.lib(), fn)
+    return f(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Hq"], args["Hkv"],
+             args["Lq"], args["Lk"], args["d"], args["scale"], args["lam"], args["causal"], args["mask"],
+             args["count"], args["stream"], ctypes.byref(opts))
+
+
+@pytest.mark.parametrize("fn", ["blasst_decode", "blasst_prefill"])
+def test_invalid_arguments_rejected_before_launch(bl, fn):
+    assert _call(bl, fn, q=None) == 1
+    assert _call(bl, fn, k=None) == 1
+    assert _call(bl, fn, v=None) == 1
+    assert _call(bl, fn, o=None) == 1
+    assert _call(bl, fn, lse=None) == 1
+    assert _call(bl, fn, B=0) == 1
+    assert _call(bl, fn, Hq=6, Hkv=4) == 1
+    assert _call(bl, fn, lam=-0.5) == 1
+    assert _call(bl, fn, lam=1.0) == 1
+    assert _call(bl, fn, lam=float("nan")) == 1
+    assert _call(bl, fn, lam=float("inf")) == 1
+    assert _call(bl, fn, scale=0.0) == 1
+    assert _call(bl, fn, scale=float("nan")) == 1
+    assert _call(bl, fn, causal=1, Lq=300, Lk=256) == 1
+    assert _call(bl, fn, q=FAKE + 8) == 1                    # misaligned
+    assert _call(bl, fn, d=64) == 2                          # head dim not built
+    assert _call(bl, fn, opts=bl.Opts(k_row_stride=130)) == 1  # stride not a multiple of 8
+    assert _call(bl, fn, opts=bl.Opts(block_n=32)) == 2
+
+
+def test_decode_unsupported_tile_and_small_workspace(bl):
+    assert _call(bl, "blasst_decode", Hq=32, Hkv=1) == 2      # G * Lq > 16
+    assert _call(bl, "blasst_decode", opts=bl.Opts(workspace=FAKE, workspace_bytes=64)) == 3
+    assert _call(bl, "blasst_decode", opts=bl.Opts(workspace=FAKE + 16, workspace_bytes=1 << 30)) == 1
+
+
+def test_calibrate_requires_gaps_and_valid_mode(bl):
+    assert _call(bl, "blasst_calibrate") == 1                 # no gaps_out
+    assert _call(bl, "blasst_calibrate", opts=bl.Opts(mode=7, gaps_out=FAKE)) == 1
+
+
+def test_old_struct_size_reads_as_defaults(bl):
+    # an older caller that only knows the first field: everything else defaults
+    o = bl.Opts(block_n=32)
+    o.struct_size = ctypes.sizeof(ctypes.c_size_t)
+    assert _call(bl, "blasst_decode", d=64, opts=o) == 2      # d=64 unsupported, block_n ignored
+
+
+def test_status_strings(bl):
+    L = bl.lib()
+    for s in range(6):
+        assert L.blasst_status_string(s)
+    assert L.blasst_last_error() is not None
+
+
+def test_calibrate_fit_exact(bl):
+    alpha, beta = 2.5, 7.0
+    Ls = np.array([8192, 16384, 32768, 65536.0])
+    s = np.array([0.3, 0.5, 0.6, 0.75])
+    lam = alpha * np.exp(beta * s) / Ls
+    a, b = bl.calibrate_fit(Ls, lam, s)
+    assert abs(a - alpha) < 1e-9 and abs(b - beta) < 1e-9
+    ao, bo = oracle.calibrate_fit(Ls, lam * (1 + 0.01 * np.arange(4)), s)
+    a2, b2 = bl.calibrate_fit(Ls, lam * (1 + 0.01 * np.arange(4)), s)
+    assert abs(a2 - ao) < 1e-9 * ao and abs(b2 - bo) < 1e-9
+
+
+def test_calibrate_fit_rejects_bad_input(bl):
+    with pytest.raises(bl.BlasstError):
+        bl.calibrate_fit([8192], [0.001], [0.5])
+    with pytest.raises(bl.BlasstError):
+        bl.calibrate_fit([8192, 8192], [0.001, 0.002], [0.5, 0.5])
+
+
+def test_calibrate_threshold_agrees_with_oracle_gaps(bl):
+    inp = planted_prefill(1, 2, 1, 2048, 32, seed=13, reading="blk", boost=True)
+    r = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.0, causal=True, BM=64, BN=32)
+    gaps = np.where(r["visited"] == 1, r["gaps"], np.nan).astype(np.float32)
+    for target in (0.2, 0.5, 0.7):
+        lam, ach = bl.calibrate_threshold(gaps, target)
+        lam_o, ach_o = oracle.threshold_for_sparsity(r["gaps"], r["visited"], target)
+        assert abs(ach - ach_o) <= 2.0 / r["n_visited"]
+        rr = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=lam, causal=True, BM=64, BN=32)
+        assert abs(rr["n_skipped"] / rr["n_visited"] - ach) <= 2.0 / r["n_visited"]
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 2, 300, 300, 1), (2, 2, 1, 1024, 1024, 1), (1, 2, 2, 100, 700, 1),
+                                   (1, 2, 2, 100, 700, 0), (1, 1, 1, 128, 128, 1)])
+def test_visited_pairs_prefill_matches_oracle(bl, shape):
+    B, Hq, Hkv, Lq, Lk, causal = shape
+    inp = random_normal(B, Hq, Hkv, Lq, Lk, 8, seed=0)
+    r = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.0, causal=bool(causal), BM=128, BN=128)
+    assert bl.visited_pairs(B, Hq, Hkv, Lq, Lk, causal, False) == r["n_visited"]
+
+
+@pytest.mark.parametrize("shape", [(2, 8, 2, 1, 1000, 0), (1, 4, 1, 3, 777, 1)])
+def test_visited_pairs_decode_matches_oracle(bl, shape):
+    B, Hq, Hkv, Lq, Lk, causal = shape
+    inp = random_normal(B, Hq, Hkv, Lq, Lk, 8, seed=0)
+    r = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.0, causal=bool(causal), is_decode=True,
+                         num_splits=4, BN=64)
+    assert bl.visited_pairs(B, Hq, Hkv, Lq, Lk, causal, True) == r["n_visited"]
+
+
+def test_visited_pairs_of_benchmark_shapes(bl):
+    # 1024-token MHA prefill: 36 pairs; 32K and 64K GQA prefill; decode 32 x 8 x 512
+    assert bl.visited_pairs(1, 1, 1, 1024, 1024, 1, False) == 36
+    assert bl.visited_pairs(1, 32, 8, 32768, 32768, 1, False) == 32 * 256 * 257 // 2
+    assert bl.visited_pairs(1, 32, 8, 65536, 65536, 1, False) == 32 * 512 * 513 // 2
+    assert bl.visited_pairs(32, 32, 8, 1, 32768, 0, True) == 32 * 8 * 512
+
+
+def test_workspace_bytes(bl):
+    rows, S, dv = 32 * 32, 16, 128
+    expect = -(-rows * S * dv * 4 // 256) * 256 + -(-rows * S * 4 // 256) * 256
+    assert bl.decode_workspace_bytes(32, 32, 1, 128, 16) == expect
+    assert bl.decode_workspace_bytes(32, 32, 1, 0, 0) == expect

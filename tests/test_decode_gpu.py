@@ -1,0 +1,185 @@
+"""GPU parity of blasst_decode (split-KV, 64-key blocks) against the fp64 oracle."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from _parity import assert_outputs_close, bf16_tensor_to_f64, compare_masks, unpack_mask
+from synth import bf16_bits, planted_decode, random_normal
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def bl():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_flashattention_tcgen05_b200 as m
+
+    m.lib()
+    return m
+
+
+def to_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True):
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    o, lse, mask, cnt = bl.decode(q, k, v, scale=inp.scale, lam=lam, causal=causal, num_splits=splits)
+    torch.cuda.synchronize()
+    B, Hq, Lq, d = inp.q.shape
+    Hkv, Lk = inp.k.shape[1], inp.k.shape[2]
+    nb = (Lk + 63) // 64
+    bits = unpack_mask(mask.cpu().numpy(), nb)
+    assert int(cnt.item()) == int(bits.sum())
+    ref = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=lam, causal=causal, is_decode=True,
+                           num_splits=splits, BN=64, tiles=tiles)
+    nd, nband = compare_masks(bits, ref, lam, tiles)
+    assert nd == 0, f"{nd} mask bits differ outside the band"
+    if not band_ok:
+        assert nband == 0
+    forced = bits.copy()
+    fr = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=lam, causal=causal, is_decode=True,
+                          num_splits=splits, BN=64, tiles=tiles, forced_skip=forced)
+    og = bf16_tensor_to_f64(o)
+    lg = lse.cpu().numpy().astype(np.float64)
+    rows = None
+    if tiles is not None:
+        G = Hq // Hkv
+        sel = np.zeros((B, Hq, Lq), bool)
+        for t in tiles:
+            b, h = divmod(int(t), Hkv)
+            sel[b, h * G:(h + 1) * G, :] = True
+        rows = sel
+    assert_outputs_close(og, lg, fr["o"], fr["lse"], rows)
+    return bits, ref
+
+
+@pytest.mark.parametrize("lam", [0.0, 1e-3, 0.05, 0.5, 0.999])
+@pytest.mark.parametrize("reading", ["blk", "lit"])
+def test_decode_gqa_small(bl, lam, reading):
+    inp = planted_decode(2, 8, 2, 64 * 37 + 13, 128, seed=21, reading=reading)
+    bits, ref = check_decode(bl, inp, lam, False, 4)
+    if lam == 0.0:
+        assert bits.sum() == 0
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.02])
+def test_decode_random_normal(bl, lam):
+    inp = random_normal(3, 4, 4, 1, 1000, 128, seed=5)
+    check_decode(bl, inp, lam, False, 16)
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.1])
+def test_decode_two_ntiles_causal(bl, lam):
+    # G * Lq = 16 rows: the wider tile variant, causal with Lq = 2
+    inp = planted_decode(1, 8, 1, 3000, 128, Lq=2, seed=3, reading="blk")
+    check_decode(bl, inp, lam, True, 3)
+
+
+def test_decode_short_cache_many_empty_splits(bl):
+    inp = planted_decode(2, 4, 1, 50, 128, seed=8, reading="lit")
+    check_decode(bl, inp, 0.3, False, 16)
+
+
+def test_decode_single_split_long(bl):
+    inp = planted_decode(1, 4, 1, 64 * 200, 128, seed=9, reading="blk")
+    bits, _ = check_decode(bl, inp, 0.05, False, 1)
+    assert bits.sum() > 0
+
+
+def test_decode_lambda_zero_matches_textbook(bl):
+    # lambda = 0 against the dense definition directly (oracle dense == brute force, pinned on CPU)
+    inp = random_normal(2, 8, 2, 1, 777, 128, seed=1)
+    check_decode(bl, inp, 0.0, False, 5)
+
+
+def _expanded_hand_case(name, BN):
+    with open(os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")) as f:
+        case = [c for c in json.load(f)["cases"] if c["name"] == name][0]
+    nkeys = len(case["key_coords"])
+    Lk = nkeys * BN
+    d = 128
+    Hq, Hkv = case["Hq"], case["Hkv"]
+    q = np.zeros((1, Hq, 1, d), np.float32)
+    for g in range(Hq):
+        q[0, g, 0, case["q_axes"][g][0] if case["mode"] == "decode" else case["q_axes"][0][0]] = 1.0
+    k = np.full((1, Hkv, Lk, d), -64.0, np.float32)
+    for j, coords in enumerate(case["key_coords"]):
+        k[0, :, j * BN, :] = -64.0
+        k[0, :, j * BN, : len(coords)] = coords
+    v = np.random.default_rng(0).standard_normal((1, Hkv, Lk, d)).astype(np.float32)
+    return case, bf16_bits(q), bf16_bits(k), bf16_bits(v)
+
+
+@pytest.mark.parametrize("name", ["one_row_four_blocks", "decode_group_two_splits", "lambda_near_one"])
+def test_decode_hand_cases_exact(bl, name):
+    # each hand key becomes a 64-key block whose other keys score -64: block maxima are exact
+    case, q, k, v = _expanded_hand_case(name, 64)
+    from synth import AttnInputs
+
+    inp = AttnInputs(q, k, v, 1.0)
+    splits = case.get("num_splits", 1)
+    for cl in case["cases_lambda"]:
+        lam = math.exp(cl["ln_lambda"]) if "ln_lambda" in cl else cl["lambda"]
+        bits, ref = check_decode(bl, inp, lam, False, splits)
+        assert bits.tolist() == cl["skip"]
+
+
+def test_decode_invalid_arguments(bl):
+    inp = random_normal(1, 4, 1, 1, 256, 128, seed=0)
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    for lam in (-0.1, 1.0, float("nan"), float("inf")):
+        with pytest.raises(bl.BlasstError) as e:
+            bl.decode(q, k, v, scale=inp.scale, lam=lam)
+        assert e.value.status == 1
+    with pytest.raises(bl.BlasstError) as e:
+        bl.decode(q, k, v, scale=-1.0, lam=0.0)
+    assert e.value.status == 1
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bl.BlasstError) as e:
+        bl.decode(q, k, v, scale=inp.scale, lam=0.0, workspace=ws)
+    assert e.value.status == 3
+
+
+def test_decode_caller_workspace_and_status_word(bl):
+    inp = planted_decode(2, 8, 2, 4000, 128, seed=2, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    nbytes = bl.decode_workspace_bytes(2, 8, 1, 128, 16)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o1, l1, m1, c1 = bl.decode(q, k, v, scale=inp.scale, lam=0.05, workspace=ws, status_word=st)
+    o2, l2, m2, c2 = bl.decode(q, k, v, scale=inp.scale, lam=0.05)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2) and torch.equal(m1, m2) and torch.equal(c1, c2)
+
+
+def test_decode_calibrate_matches_decode_masks(bl):
+    inp = planted_decode(2, 8, 2, 5000, 128, seed=4, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    gaps, mc, cc = bl.calibrate(q, k, scale=inp.scale, lam=0.05, mode="decode", num_splits=4)
+    _, _, md, cd = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=4)
+    torch.cuda.synchronize()
+    assert torch.equal(mc, md) and torch.equal(cc, cd)
+    ref = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.05, causal=False, is_decode=True,
+                           num_splits=4, BN=64)
+    g = gaps.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(ref["gaps"])
+    assert np.array_equal(np.isinf(g), np.isinf(ref["gaps"]))
+    assert np.max(np.abs(g[fin] - ref["gaps"][fin])) < 1e-3
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("lam", [0.0, 0.05])
+def test_decode_full_size_sampled(bl, lam):
+    # batch 32, Hq 32 / Hkv 8, 32768-key cache, 16 splits: the benchmarked launch; oracle on sampled tiles
+    inp = planted_decode(32, 32, 8, 32768, 128, seed=3, reading="blk")
+    rng = np.random.default_rng(0)
+    tiles = np.sort(rng.choice(32 * 8, 12, replace=False))
+    check_decode(bl, inp, lam, False, 16, tiles=tiles)

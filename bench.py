@@ -1,0 +1,586 @@
+#!/usr/bin/env python
+"""Benchmark of the BLASST hot path on B200 (libblasst.so through its C ABI).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+Headline workload: GQA prefill with the Llama-3.1-8B attention shape (B=1,
+Hq=32, Hkv=8, d=128, Lq=Lk=32768, causal, bf16) at the lambda that gives ~75%
+block sparsity; one step = one prefill call.  Effective work per call counts
+Q.K^T on every visited (tile, block) pair plus P.V on kept pairs, 2*128^3
+FLOP each.  The same run also measures (the "sweep"): prefill at ~0/50/75%
+sparsity and split-KV GQA decode (batch 32, Hq=32, Hkv=8, 32768-key cache,
+16 splits) at ~0/50/75%, whose effective bytes are all K bytes + kept V bytes
++ q/o/lse.  Lambdas come from one calibration pass (decision-only kernel)
+per workload: a pair is skipped iff its gap < ln(lambda), so the quantiles of
+the gaps give the lambda for each target.
+
+Inputs: seeded planted-direction generator ("blk" reading: planted logit +8,
+5% heavy keys in 64-key runs, +2 local boost), bf16.  L2 is flushed (256 MiB
+write) before every timed launch; timing uses CUDA events on the launching
+stream.  The CPU baseline is the fp64 oracle timed on the host cores over a
+bounded sample of query tiles of the same workload.
+
+With N > 1 (torchrun), every rank runs an independent replica of the
+workload on its own GPU (the problems are independent; no data-path
+collective) and the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill eff. TFLOP/s & decode eff. HBM GB/s at 0/50/75% sparsity (1×B200)"
+FLOP_PER_PAIR = 2 * 128 * 128 * 128
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, Hq=32, Hkv=8, L=32768, d=128,
+               causal=True, seed=2)
+DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk=32768, d=128, splits=16, seed=3)
+QUICK_PREFILL = dict(PREFILL, workload="prefill GQA 4K (quick)", L=4096)
+QUICK_DECODE = dict(DECODE, workload="decode GQA 4K cache (quick)", B=4, Lk=4096)
+# profiling size: inputs larger than L2 (126 MB) but a few GB at most on the device
+MEDIUM_PREFILL = dict(PREFILL, workload="prefill GQA 8K (profiling size)", L=8192)
+MEDIUM_DECODE = dict(DECODE, workload="decode GQA 32K cache, batch 8 (profiling size)", B=8)
+SIZES = {"full": (PREFILL, DECODE), "medium": (MEDIUM_PREFILL, MEDIUM_DECODE), "quick": (QUICK_PREFILL, QUICK_DECODE)}
+TARGETS = (0.0, 0.5, 0.75)
+
+
+# --------------------------------------------------------------------------- utils
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_profile_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d.get(kernel_key)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons, polled through NVML every
+    few milliseconds while the timed region runs (read-only queries)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.windows = []
+        self.stop_flag = False
+        self.h = None
+        self.max_mhz = None
+        try:
+            import pynvml as nv
+            import torch
+
+            nv.nvmlInit()
+            self.nv = nv
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = nv.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+
+    def start(self):
+        if self.h is None:
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.time(), mhz, r))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        self.stop_flag = True
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvml unavailable"}
+        self.t.join(timeout=2)
+        inside = [s for s in self.samples if any(a <= s[0] <= b for a, b in self.windows)]
+        use = inside or self.samples
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
+        reasons = set()
+        for _, _, r in use:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(use), "in_timed_region": bool(inside), "source": "nvml"}
+
+
+def to_dev(a, device):
+    import numpy as np
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def to_pinned(a):
+    import numpy as np
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+
+# --------------------------------------------------------------------- workloads
+class Prefill:
+    kind = "prefill"
+    unit = "TFLOP/s"
+    bound = "tensor"
+
+    def __init__(self, cfg, device):
+        import synth
+
+        self.cfg = cfg
+        self.device = device
+        c = cfg
+        self.inp = synth.planted_prefill(c["B"], c["Hq"], c["Hkv"], c["L"], c["d"], seed=c["seed"], reading="blk")
+        self.q, self.k, self.v = (to_dev(x, device) for x in (self.inp.q, self.inp.k, self.inp.v))
+        import torch
+
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:3], dtype=torch.float32, device=device)
+        import block_sparse_flashattention_tcgen05_b200 as bl
+
+        self.bl = bl
+        self.visited = bl.visited_pairs(c["B"], c["Hq"], c["Hkv"], c["L"], c["L"], True, False)
+        self.launches = 1
+
+    def calibrate(self):
+        gaps, _, _ = self.bl.calibrate(self.q, self.k, scale=self.inp.scale, causal=True, mode="prefill")
+        return gaps.cpu().numpy()
+
+    def call(self, lam, stream=None):
+        return self.bl.prefill(self.q, self.k, self.v, scale=self.inp.scale, lam=lam, causal=True, o=self.o,
+                               lse=self.lse, skip_mask=False, skip_count=self.count, stream=stream)
+
+    def work(self, skipped):
+        kept = self.visited - skipped
+        return FLOP_PER_PAIR * (self.visited + kept)
+
+    def rate(self, work, ms):
+        return work / (ms * 1e-3) / 1e12
+
+    def host_bytes(self):
+        return (self.inp.q.nbytes + self.inp.k.nbytes + self.inp.v.nbytes,
+                self.inp.q.nbytes + self.lse.numel() * 4)
+
+    def e2e_call(self, lam, hq, hk, hv, ho, hl):
+        self.q.copy_(hq, non_blocking=True)
+        self.k.copy_(hk, non_blocking=True)
+        self.v.copy_(hv, non_blocking=True)
+        self.call(lam)
+        ho.copy_(self.o, non_blocking=True)
+        hl.copy_(self.lse, non_blocking=True)
+
+
+class Decode:
+    kind = "decode"
+    unit = "GB/s"
+    bound = "hbm"
+
+    def __init__(self, cfg, device):
+        import synth
+
+        self.cfg = cfg
+        self.device = device
+        c = cfg
+        self.inp = synth.planted_decode(c["B"], c["Hq"], c["Hkv"], c["Lk"], c["d"], seed=c["seed"], reading="blk")
+        self.q, self.k, self.v = (to_dev(x, device) for x in (self.inp.q, self.inp.k, self.inp.v))
+        import torch
+
+        import block_sparse_flashattention_tcgen05_b200 as bl
+
+        self.bl = bl
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:3], dtype=torch.float32, device=device)
+        self.ws = torch.empty(bl.decode_workspace_bytes(c["B"], c["Hq"], 1, 128, c["splits"]), dtype=torch.uint8,
+                              device=device)
+        self.visited = bl.visited_pairs(c["B"], c["Hq"], c["Hkv"], 1, c["Lk"], False, True)
+        self.launches = 2
+
+    def calibrate(self):
+        gaps, _, _ = self.bl.calibrate(self.q, self.k, scale=self.inp.scale, causal=False, mode="decode",
+                                       num_splits=self.cfg["splits"])
+        return gaps.cpu().numpy()
+
+    def call(self, lam, stream=None):
+        return self.bl.decode(self.q, self.k, self.v, scale=self.inp.scale, lam=lam, num_splits=self.cfg["splits"],
+                              o=self.o, lse=self.lse, skip_mask=False, skip_count=self.count, workspace=self.ws,
+                              stream=stream)
+
+    def work(self, skipped):
+        c = self.cfg
+        blk_bytes = 64 * c["d"] * 2
+        k_bytes = c["B"] * c["Hkv"] * c["Lk"] * c["d"] * 2
+        kept = self.visited - skipped
+        qo = self.inp.q.nbytes * 2 + self.lse.numel() * 4
+        return k_bytes + kept * blk_bytes + qo
+
+    def rate(self, work, ms):
+        return work / (ms * 1e-3) / 1e9
+
+    def host_bytes(self):
+        return (self.inp.q.nbytes + self.inp.k.nbytes + self.inp.v.nbytes,
+                self.inp.q.nbytes + self.lse.numel() * 4)
+
+    def e2e_call(self, lam, hq, hk, hv, ho, hl):
+        self.q.copy_(hq, non_blocking=True)
+        self.k.copy_(hk, non_blocking=True)
+        self.v.copy_(hv, non_blocking=True)
+        self.call(lam)
+        ho.copy_(self.o, non_blocking=True)
+        hl.copy_(self.lse, non_blocking=True)
+
+
+def lambdas_for_targets(wl, gaps):
+    out = {}
+    for t in TARGETS:
+        if t == 0.0:
+            out[t] = (0.0, 0.0)
+            continue
+        lam, ach = wl.bl.calibrate_threshold(gaps, t)
+        if ach + 0.02 < t:  # unreachable target: the highest reachable sparsity
+            lam, ach = wl.bl.calibrate_threshold(gaps, 1.0)
+        out[t] = (lam, ach)
+    return out
+
+
+def timed_launches(wl, lam, steps, warmup, flush, sampler=None):
+    """Per-launch device times (ms) with CUDA events on the launching stream, L2 flushed before each."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    wl.count = torch.zeros(1, dtype=torch.int64, device=wl.device)
+    for _ in range(warmup):
+        wl.call(lam)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0 = time.time()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        wl.call(lam)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if sampler:
+        sampler.mark(t0, t1)
+    ms = [a.elapsed_time(b) for a, b in ev]
+    skipped = int(wl.count.item())
+    return ms, skipped
+
+
+def e2e_measure(wl, lam, steps, warmup):
+    import torch
+
+    hq, hk, hv = to_pinned(wl.inp.q), to_pinned(wl.inp.k), to_pinned(wl.inp.v)
+    ho = torch.empty(wl.o.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
+    wl.count = torch.zeros(1, dtype=torch.int64, device=wl.device)
+    for _ in range(max(1, warmup)):
+        wl.e2e_call(lam, hq, hk, hv, ho, hl)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        wl.e2e_call(lam, hq, hk, hv, ho, hl)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    skipped = int(wl.count.item())
+    hb, db = wl.host_bytes()
+    return ms, skipped, hb, db
+
+
+# ------------------------------------------------------------------ CPU baseline
+def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of query tiles.
+
+    Returns dict(value, unit, cores, kind, sample)."""
+    import numpy as np
+
+    import oracle
+    import synth
+
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    rng = np.random.default_rng(seed_tiles)
+    if wl_kind == "prefill":
+        c = cfg
+        inp = synth.planted_prefill(c["B"], c["Hq"], c["Hkv"], c["L"], c["d"], seed=c["seed"], reading="blk")
+        nq = c["L"] // 128
+        n_tiles = c["B"] * c["Hq"] * nq
+        # tiles from the last quarter of the sequence (long rows); count grows until the budget is used
+        cand = [t for t in range(n_tiles) if (t % nq) >= nq * 3 // 4]
+        rng.shuffle(cand)
+        kw = dict(scale=inp.scale, causal=True)
+        units = lambda r: FLOP_PER_PAIR * (r["n_visited"] * 2 - r["n_skipped"]) / 1e12  # noqa: E731
+        unit = "TFLOP/s"
+    else:
+        c = cfg
+        inp = synth.planted_decode(c["B"], c["Hq"], c["Hkv"], c["Lk"], c["d"], seed=c["seed"], reading="blk")
+        cand = list(range(c["B"] * c["Hkv"]))
+        rng.shuffle(cand)
+        kw = dict(scale=inp.scale, causal=False, is_decode=True, num_splits=c["splits"])
+        blk = 64 * c["d"] * 2
+        keyb = c["Lk"] * c["d"] * 2
+        n_tiles = len(cand)
+
+        def units(r):
+            return (r["_tiles"] * keyb + (r["n_visited"] - r["n_skipped"]) * blk) / 1e9
+        unit = "GB/s"
+    # calibrate lambda on the first tiles (their own gaps), then time
+    n = max(1, min(len(cand), cores))
+    t0 = time.time()
+    r0 = oracle.attention(inp.q, inp.k, inp.v, lam=0.0, tiles=cand[:n], **kw)
+    dt = time.time() - t0
+    lam, _ = oracle.threshold_for_sparsity(r0["gaps"][cand[:n]], r0["visited"][cand[:n]], lam_target)
+    n = int(max(1, min(len(cand), n * budget_s / max(dt, 1e-3))))
+    tiles = cand[:n]
+    t0 = time.time()
+    r = oracle.attention(inp.q, inp.k, inp.v, lam=lam, tiles=tiles, **kw)
+    dt = time.time() - t0
+    r["_tiles"] = len(tiles)
+    return dict(value=units(r) / dt, unit=unit, cores=cores, kind="oracle",
+                sample=f"{len(tiles)} of {n_tiles} query tiles "
+                       f"({'last quarter of the sequence' if wl_kind == 'prefill' else 'whole KV heads'}), "
+                       f"lambda={lam:.4g} for ~{lam_target:.0%} sparsity on the sample, {dt:.1f} s",
+                seconds=dt)
+
+
+# -------------------------------------------------------------------------- main
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def aggregate(units_local, seconds_local, world):
+    """Whole-job throughput: units over all ranks / max over ranks of the time."""
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([seconds_local], dtype=torch.float64, device=dev)
+        u = torch.tensor([units_local], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+        return u.item() / t.item(), t.item()
+    return units_local / seconds_local, seconds_local
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl_kind = "prefill" if args.workload == "prefill" else "decode"
+    cfg = SIZES[args.size][0] if wl_kind == "prefill" else SIZES[args.size][1]
+    per_step = []
+    vals = []
+    budget = float(os.environ.get("BLASST_REF_STEP_SECONDS", "8"))
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(wl_kind, cfg, budget_s=budget, seed_tiles=i)
+        if i >= args.warmup:
+            per_step.append(r["seconds"])
+            vals.append(r["value"])
+    value = statistics.mean(vals)
+    unit = "TFLOP/s" if wl_kind == "prefill" else "GB/s"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "lambda_target": 0.75, "reading": "blk"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": r["cores"], "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--workload", choices=["prefill", "decode"], default="prefill")
+    ap.add_argument("--size", choices=sorted(SIZES), default="full",
+                    help="full = the benchmark shapes; medium = profiling size; quick = smoke-testing the bench")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    import torch
+
+    import block_sparse_flashattention_tcgen05_b200 as bl
+
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    notes = []
+
+    pcfg, dcfg = SIZES[args.size]
+    headline_kind = args.workload
+    wls = {}
+    try:
+        wls["prefill"] = Prefill(pcfg, dev)
+        wls["prefill"].count = torch.zeros(1, dtype=torch.int64, device=dev)
+        wls["prefill"].call(0.0)
+        torch.cuda.synchronize()
+    except bl.BlasstError as e:
+        if e.status != 2:
+            raise
+        wls.pop("prefill", None)
+        notes.append("prefill kernel not available in this build; headline falls back to decode")
+        headline_kind = "decode"
+    if headline_kind == "decode" or not args.no_sweep:
+        wls["decode"] = Decode(dcfg, dev)
+
+    lams = {k: lambdas_for_targets(w, w.calibrate()) for k, w in wls.items()}
+
+    # ---- headline: the ~75% point of the headline workload
+    wl = wls[headline_kind]
+    lam75, ach75 = lams[headline_kind][0.75]
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms, skipped = timed_launches(wl, lam75, args.steps, args.warmup, flush, sampler)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    work = wl.work(skipped)
+    ms_mean = statistics.mean(ms)
+    value, t_max = aggregate(work * args.steps, sum(ms) * 1e-3, world)
+    value = value / (1e12 if wl.unit == "TFLOP/s" else 1e9)
+    achieved = wl.rate(work, ms_mean)
+    if wl.bound == "tensor":
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peak_src} bf16 burst", "traffic": load_profile_traffic("prefill")}
+    else:
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": f"{peak_src} copy bandwidth", "traffic": load_profile_traffic("decode")}
+
+    # ---- sweep: 0/50/75% on both workloads, speedup over lambda = 0
+    sweep = {}
+    if not args.no_sweep:
+        for kind, w in wls.items():
+            rows = {}
+            base = None
+            for t in TARGETS:
+                lam, ach = lams[kind][t]
+                ms_t, sk = timed_launches(w, lam, max(5, args.steps // 2), 3, flush)
+                med = statistics.median(ms_t)
+                r = w.rate(w.work(sk), med)
+                if t == 0.0:
+                    base = med
+                pk = peaks["bf16_tflops"] if w.bound == "tensor" else peaks["hbm_gbs"]
+                rows[f"{int(t * 100)}%"] = {
+                    "lambda": lam, "a=lambda*L": lam * (w.cfg.get("L") or w.cfg.get("Lk")),
+                    "sparsity": sk / w.visited, "ms": med, "value": r, "unit": w.unit,
+                    "frac_of_measured_peak": r / pk, "speedup_vs_lambda0": base / med}
+            sweep[kind] = rows
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e_ms, e_sk, hb, db = e2e_measure(wl, lam75, max(3, args.steps // 4), 1)
+        e_val, _ = aggregate(wl.work(e_sk), e_ms * 1e-3, world)
+        e2e = {"value": e_val / (1e12 if wl.unit == "TFLOP/s" else 1e9), "unit": wl.unit, "h2d_bytes_per_step": hb,
+               "d2h_bytes_per_step": db, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(headline_kind, wl.cfg, budget_s=float(os.environ.get("BLASST_CPU_SECONDS", "12")))
+        cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    cfgd = {"workload": wl.cfg["workload"], "lambda": lam75, "target_sparsity": 0.75, "achieved_sparsity":
+            skipped / wl.visited, "visited_pairs": wl.visited, "reading": "blk",
+            "l2": "flushed (256 MiB write) before every timed launch"}
+    for k in ("B", "Hq", "Hkv", "L", "Lk", "d", "splits"):
+        if k in wl.cfg:
+            cfgd[k] = wl.cfg[k]
+    line = {
+        "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfgd,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": wl.launches * args.steps,
+        "clocks": clocks, "sweep": sweep, "notes": notes,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -45,6 +45,7 @@ struct DecodeSmemTail {
     uint64_t v_empty[8];
     float red[2][kConsumerWarps][16];
     float lred[kConsumerWarps][16];
+    float rred[kConsumerWarps][16];
     float mfin[16];
     int dec_count;
     int abort;
@@ -182,10 +183,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int c = 0; c < NC; c++) Mall[c] = -CUDART_INF_F;
     float o_acc[CALIB ? 1 : 8][NT][4];
-    float lsum[NT][2];
+    // lsum: exact fp32 partial row sums (for lse); lrnd: sums of the bf16-rounded
+    // P that P.V uses (normalises O exactly)
+    float lsum[NT][2], lrnd[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; nt++) {
         lsum[nt][0] = lsum[nt][1] = 0.f;
+        lrnd[nt][0] = lrnd[nt][1] = 0.f;
         if (!CALIB)
 #pragma unroll
             for (int mt = 0; mt < 8; mt++)
@@ -318,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 const float alpha = (mnew == NEG_INF) ? 1.f : ex2(mold - mnew);
                 lsum[nt][e] *= alpha;
+                lrnd[nt][e] *= alpha;
 #pragma unroll
                 for (int mt = 0; mt < 8; mt++) {
                     o_acc[mt][nt][e] *= alpha;
@@ -327,8 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pv[2 + e] = s[nt][2 + e] == NEG_INF ? 0.f : ex2(s[nt][2 + e] - mnew);
                 lsum[nt][e] += pv[e] + pv[2 + e];
             }
-            pb[nt][0] = movmatrix_t(pack_bf16x2(pv[0], pv[1]));
-            pb[nt][1] = movmatrix_t(pack_bf16x2(pv[2], pv[3]));
+            const uint32_t lo = pack_bf16x2(pv[0], pv[1]);
+            const uint32_t hi = pack_bf16x2(pv[2], pv[3]);
+            lrnd[nt][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
+            lrnd[nt][1] += __uint_as_float(lo & 0xFFFF0000u) + __uint_as_float(hi & 0xFFFF0000u);
+            pb[nt][0] = movmatrix_t(lo);
+            pb[nt][1] = movmatrix_t(hi);
         }
 #pragma unroll
         for (int c = 0; c < NC; c++) Mall[c] = Mn[c];
@@ -367,11 +376,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int nt = 0; nt < NT; nt++) {
 #pragma unroll
         for (int e = 0; e < 2; e++) {
-            float l = lsum[nt][e];
-            l += __shfl_xor_sync(0xffffffffu, l, 4);
-            l += __shfl_xor_sync(0xffffffffu, l, 8);
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
-            if (g4 == 0) tl->lred[warp][nt * 8 + 2 * t4 + e] = l;
+            float l = lsum[nt][e], lr = lrnd[nt][e];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                l += __shfl_xor_sync(0xffffffffu, l, o);
+                lr += __shfl_xor_sync(0xffffffffu, lr, o);
+            }
+            if (g4 == 0) {
+                tl->lred[warp][nt * 8 + 2 * t4 + e] = l;
+                tl->rred[warp][nt * 8 + 2 * t4 + e] = lr;
+            }
         }
 #pragma unroll
         for (int mt = 0; mt < 8; mt++) {
@@ -392,14 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = threadIdx.x;  // dv index 0..127
     const int S = p.num_splits;
     for (int c = 0; c < p.R; c++) {
-        float l = 0.f, o = 0.f;
+        float l = 0.f, lr = 0.f, o = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; w++) {
             l += tl->lred[w][c];
+            lr += tl->rred[w][c];
             o += obuf[(w * 128 + x) * NC + c];
         }
         const size_t row = (size_t)(qrow0 + c) * S + split;
-        p.part_o[row * 128 + x] = l > 0.f ? o / l : 0.f;
+        p.part_o[row * 128 + x] = lr > 0.f ? o / lr : 0.f;
         if (x == 0) p.part_lse[row] = l > 0.f ? (tl->mfin[c] + __log2f(l)) * 0.69314718055994531f : NEG_INF;
     }
 }

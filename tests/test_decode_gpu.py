@@ -103,7 +103,8 @@ def _expanded_hand_case(name, BN):
     with open(os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")) as f:
         case = [c for c in json.load(f)["cases"] if c["name"] == name][0]
     nkeys = len(case["key_coords"])
-    Lk = nkeys * BN
+    bn0 = case["BN"]  # keys per block in the hand case; each block becomes one BN-key block
+    Lk = (nkeys // bn0) * BN
     d = 128
     Hq, Hkv = case["Hq"], case["Hkv"]
     q = np.zeros((1, Hq, 1, d), np.float32)
@@ -111,8 +112,7 @@ def _expanded_hand_case(name, BN):
         q[0, g, 0, case["q_axes"][g][0] if case["mode"] == "decode" else case["q_axes"][0][0]] = 1.0
     k = np.full((1, Hkv, Lk, d), -64.0, np.float32)
     for j, coords in enumerate(case["key_coords"]):
-        k[0, :, j * BN, :] = -64.0
-        k[0, :, j * BN, : len(coords)] = coords
+        k[0, :, (j // bn0) * BN + j % bn0, : len(coords)] = coords
     v = np.random.default_rng(0).standard_normal((1, Hkv, Lk, d)).astype(np.float32)
     return case, bf16_bits(q), bf16_bits(k), bf16_bits(v)
 

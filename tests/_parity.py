@@ -51,13 +51,28 @@ def compare_masks(gpu_bits, ref, lam, tiles=None):
     return int(np.count_nonzero(diff & ~band)), int(np.count_nonzero(band))
 
 
-def assert_outputs_close(o_gpu, lse_gpu, o_ref, lse_ref, rows=None):
-    """o_gpu/lse_gpu numpy f64 arrays; rows: optional boolean/index selection."""
+def assert_outputs_close(o_gpu, lse_gpu, o_ref, lse_ref, rows=None, one_hot=False):
+    """o_gpu/lse_gpu numpy f64 arrays; rows: optional boolean/index selection.
+
+    one_hot=True is for the hand-built cases whose softmax rows are nearly
+    one-hot, so |O| ~ |v| ~ 1: there bf16 output rounding alone averages about
+    a quarter ulp (~2e-3 in [1, 2)) and a 1e-3 mean bound cannot hold.  Each
+    element must then be within one bf16 ulp of the fp64 value plus the
+    rounding of P to bf16 (2^-9 relative, times max |v| <= 4), and max-abs
+    stays <= 1e-2.
+    """
     if rows is not None:
         o_gpu, o_ref = o_gpu[rows], o_ref[rows]
         lse_gpu, lse_ref = lse_gpu[rows], lse_ref[rows]
     err = np.abs(o_gpu - o_ref)
     assert np.all(np.isfinite(o_gpu)), "non-finite output"
+    if one_hot:
+        mag = np.maximum(np.abs(o_ref), 2.0 ** -14)
+        ulp = np.exp2(np.floor(np.log2(mag)) - 7)
+        assert np.all(err <= ulp + 4 * 2.0 ** -9), "element off by more than 1 ulp + P rounding"
+        assert err.max() <= O_MAX_ABS, f"max-abs {err.max():.3e}"
+        assert np.abs(lse_gpu - lse_ref).max() <= LSE_ABS
+        return float(err.max()), float(err.mean()), float(np.abs(lse_gpu - lse_ref).max())
     big = np.abs(o_ref) >= 4.0
     if np.any(big):
         # beyond |O| = 4 half a bf16 ulp exceeds the absolute bound: 1 ulp there

@@ -28,7 +28,7 @@ def to_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True):
+def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True, one_hot=False):
     q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
     o, lse, mask, cnt = bl.decode(q, k, v, scale=inp.scale, lam=lam, causal=causal, num_splits=splits)
     torch.cuda.synchronize()
@@ -56,7 +56,7 @@ def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True):
             b, h = divmod(int(t), Hkv)
             sel[b, h * G:(h + 1) * G, :] = True
         rows = sel
-    assert_outputs_close(og, lg, fr["o"], fr["lse"], rows)
+    assert_outputs_close(og, lg, fr["o"], fr["lse"], rows, one_hot=one_hot)
     return bits, ref
 
 
@@ -127,7 +127,7 @@ def test_decode_hand_cases_exact(bl, name):
     splits = case.get("num_splits", 1)
     for cl in case["cases_lambda"]:
         lam = math.exp(cl["ln_lambda"]) if "ln_lambda" in cl else cl["lambda"]
-        bits, ref = check_decode(bl, inp, lam, False, splits)
+        bits, ref = check_decode(bl, inp, lam, False, splits, one_hot=True)
         assert bits.tolist() == cl["skip"]
 
 

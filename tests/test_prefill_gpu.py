@@ -28,7 +28,7 @@ def to_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def check_prefill(bl, inp, lam, causal, tiles=None):
+def check_prefill(bl, inp, lam, causal, tiles=None, one_hot=False):
     q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse, mask, cnt = bl.prefill(q, k, v, scale=inp.scale, lam=lam, causal=causal, status_word=st)
@@ -55,7 +55,7 @@ def check_prefill(bl, inp, lam, causal, tiles=None):
             b, h = divmod(bh, Hq)
             sel[b, h, qt * 128:(qt + 1) * 128] = True
         rows = sel
-    assert_outputs_close(og, lg, fr["o"], fr["lse"], rows)
+    assert_outputs_close(og, lg, fr["o"], fr["lse"], rows, one_hot=one_hot)
     return bits, ref
 
 
@@ -125,7 +125,7 @@ def test_prefill_hand_cases_exact(bl, name):
     case, inp = _expanded_hand_case(name)
     for cl in case["cases_lambda"]:
         lam = math.exp(cl["ln_lambda"]) if "ln_lambda" in cl else cl["lambda"]
-        bits, _ = check_prefill(bl, inp, lam, False)
+        bits, _ = check_prefill(bl, inp, lam, False, one_hot=True)
         assert bits.tolist() == cl["skip"]
 
 

@@ -11,7 +11,7 @@ import ctypes
 import os
 
 __all__ = [
-    "BlasstError", "lib", "prefill", "decode", "calibrate", "calibrate_fit", "calibrate_threshold",
+    "BlasstError", "lib", "prefill", "decode", "decode_noalloc", "calibrate", "calibrate_fit", "calibrate_threshold",
     "visited_pairs", "decode_workspace_bytes", "mask_words", "Opts", "STATUS",
 ]
 
@@ -71,7 +71,7 @@ def lib() -> ctypes.CDLL:
             raise ImportError(f"{LIB_PATH} is missing: build it with "
                               "`python -m block_sparse_flashattention_tcgen05_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
-        for name in ("blasst_prefill", "blasst_decode", "blasst_calibrate"):
+        for name in ("blasst_prefill", "blasst_decode", "blasst_calibrate", "blasst_decode_noalloc"):
             f = getattr(L, name)
             f.restype = ctypes.c_int
             f.argtypes = _ATTN_ARGS
@@ -95,7 +95,7 @@ def lib() -> ctypes.CDLL:
 
 def _check(rc: int, what: str):
     if rc != 0:
-        detail = lib().blasst_last_error().decode() if rc == 4 else ""
+        detail = lib().blasst_last_error().decode() if rc in (3, 4) else ""
         raise BlasstError(rc, what, detail)
 
 
@@ -194,6 +194,33 @@ def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=
                  want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hkv,
                  n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=dv)
     return o, lse, m, c
+
+
+def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=None, skip_mask=True,
+                   skip_count=True, status_word=None, stream=None):
+    """Same as decode(), through blasst_decode_noalloc: the library allocates
+    nothing (split partials in its fixed device array).  Output tensors that
+    are not passed are created here, by the caller side of the interface."""
+    import torch
+
+    _dev_tensor(q, "q"), _dev_tensor(k, "k"), _dev_tensor(v, "v")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    opts = Opts(num_splits=num_splits, dv=dv,
+                status_word=None if status_word is None else status_word.data_ptr())
+    nb = (Lk + 63) // 64
+    m, c = _attn("blasst_decode_noalloc", q, k, v, scale=scale, lam=lam, causal=causal, o=o, lse=lse,
+                 want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hkv,
+                 n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=dv)
+    return o, lse, m, c
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=16, skip_mask=True,

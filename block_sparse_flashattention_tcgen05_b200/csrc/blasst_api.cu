@@ -15,8 +15,12 @@
 using namespace blasst;
 
 namespace {
-
 thread_local char g_last_error[256] = "";
+}  // namespace
+
+void blasst::set_last_error(const char *msg) { std::snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+
+namespace {
 
 blasst_status cuda_fail(cudaError_t e, const char *where) {
     std::snprintf(g_last_error, sizeof g_last_error, "%s: %s", where, cudaGetErrorString(e));

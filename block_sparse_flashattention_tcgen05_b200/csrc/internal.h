@@ -53,6 +53,9 @@ struct PrefillParams {
     float thr_log2;
 };
 
+// Records the text returned by blasst_last_error() for this thread.
+void set_last_error(const char *msg);
+
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
                           int nt, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t stream);

@@ -155,6 +155,37 @@ BLASST_API blasst_status blasst_calibrate_fit(const double *L, const double *lam
 BLASST_API blasst_status blasst_calibrate_threshold(const float *gaps, long long n, double target_sparsity,
                                          double *lambda_out, double *achieved_out);
 
+/*
+ * Decode that allocates nothing.  The paper has no counterpart: this is a
+ * deployment variant of blasst_decode for callers that cannot allocate device
+ * memory while they run -- e.g. an engine that reserves (nearly) all device
+ * memory for its own pool up front, so any further cudaMalloc/cudaMallocAsync
+ * fails or fragments it, or a latency-critical loop where an allocation or a
+ * free could stall the device.  Same arguments, results and errors as
+ * blasst_decode, except:
+ *   - the split partials live in one fixed device array owned by the library
+ *     (BLASST_NOALLOC_SCRATCH_BYTES per GPU, held from library load until
+ *     process exit); opts->workspace must be NULL;
+ *   - calls needing more than BLASST_NOALLOC_SCRATCH_BYTES of partials
+ *     (blasst_decode_workspace_bytes) return BLASST_ERR_WORKSPACE with the
+ *     sizes in blasst_last_error();
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, which loads the module on that device); make
+ *     that first call before any stream capture;
+ *   - every call on a device shares the one array and it keeps the last
+ *     call's contents (nothing in it needs clearing: each call writes every
+ *     partial it reads), so calls that may overlap on the GPU -- on different
+ *     streams or from different host threads -- race: serialise them.
+ * It calls no cudaMalloc, cudaMallocAsync, cudaFree or other allocating
+ * routine.
+ */
+#define BLASST_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                               int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                                               float lambda, int causal, uint32_t *skip_mask,
+                                               unsigned long long *skip_count, void *stream,
+                                               const blasst_opts *opts);
+
 /* Bytes of decode workspace for these sizes (num_splits 0 -> 16, dv 0 -> 128). */
 BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_splits);
 

@@ -48,7 +48,7 @@ DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk
 QUICK_PREFILL = dict(PREFILL, workload="prefill GQA 4K (quick)", L=4096)
 QUICK_DECODE = dict(DECODE, workload="decode GQA 4K cache (quick)", B=4, Lk=4096)
 # profiling size: inputs larger than L2 (126 MB) but a few GB at most on the device
-MEDIUM_PREFILL = dict(PREFILL, workload="prefill GQA 8K (profiling size)", L=8192)
+MEDIUM_PREFILL = dict(PREFILL, workload="prefill GQA 16K (profiling size)", L=16384)
 MEDIUM_DECODE = dict(DECODE, workload="decode GQA 32K cache, batch 8 (profiling size)", B=8)
 SIZES = {"full": (PREFILL, DECODE), "medium": (MEDIUM_PREFILL, MEDIUM_DECODE), "quick": (QUICK_PREFILL, QUICK_DECODE)}
 TARGETS = (0.0, 0.5, 0.75)

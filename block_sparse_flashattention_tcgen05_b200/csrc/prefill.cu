@@ -173,17 +173,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16(128, 128, 0);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 128, 1);
-            const uint32_t s_col[2] = {tmem + 0, tmem + 128};
-            const uint32_t o_col[2] = {tmem + 256, tmem + 384};
             int n_pv[2] = {0, 0};
             bool ok = mbar_wait(&tl->q_full, 0, &tl->abort);
             auto issue_s = [&](int t, int j) {
                 const uint32_t qa = smem_addr(sq + t * kTileBytes);
                 const uint32_t ka = smem_addr(sk + (j % kStages) * kTileBytes);
+                const uint32_t s_col = tmem + (uint32_t)t * 128u;
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++) {
                     const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    umma_ss(s_col[t], umma_desc_sw128(qa + off, 16), umma_desc_sw128(ka + off, 16), idesc_s, kk > 0);
+                    umma_ss(s_col, umma_desc_sw128(qa + off, 16), umma_desc_sw128(ka + off, 16), idesc_s, kk > 0);
                 }
                 umma_commit(&tl->s_full[t]);
             };
@@ -199,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = j % kStages;
                 bool v_waited = false;
                 bool k_next_waited = false;
+#pragma unroll
                 for (int t = 0; t < 2; t++) {
                     if (j > jmax[t]) continue;
                     if (!mbar_wait(&tl->p_full[t], j & 1, &tl->abort)) {
@@ -218,9 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             v_waited = true;
                         }
                         const uint32_t va = smem_addr(sv + st * kTileBytes);
+                        const uint32_t s_col = tmem + (uint32_t)t * 128u;
+                        const uint32_t o_col = tmem + 256u + (uint32_t)t * 128u;
 #pragma unroll
                         for (int kk = 0; kk < 8; kk++)
-                            umma_ts(o_col[t], s_col[t] + kk * 8, umma_desc_sw128(va + kk * 2048, kBoxBytes), idesc_pv,
+                            umma_ts(o_col, s_col + kk * 8, umma_desc_sw128(va + kk * 2048, kBoxBytes), idesc_pv,
                                     (n_pv[t] > 0 || kk > 0) ? 1u : 0u);
                         umma_commit(&tl->o_done[t]);
                         n_pv[t]++;
@@ -267,14 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp & 3;                 // TMEM lane quadrant
         const int row = threadIdx.x & 127;       // tile row == TMEM lane
         const int bar_id = 1 + t;
-        const int qpos = q0[t] + row;
+        const int q0t = pair * 256 + t * 128;
+        const int jmaxt = last_block(p, q0t);
+        const int qpos = q0t + row;
         const bool valid_row = qpos < p.Lq;
         const int last_key = !valid_row ? -1 : (p.causal ? qpos + p.Lk - p.Lq : p.Lk - 1);
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + (t ? 128u : 0u);
         const uint32_t o_addr = tmem + lane_off + (t ? 384u : 256u);
         const float NEG_INF = -CUDART_INF_F;
-        const size_t tile_idx = ((size_t)b * p.Hq + hq) * p.n_qtiles + (q0[t] >> 7);
+        const size_t tile_idx = ((size_t)b * p.Hq + hq) * p.n_qtiles + (q0t >> 7);
         // l: exact fp32 row sum (for lse); lr: sum of the bf16-rounded P that P.V
         // uses (normalises O, so a dominant key reproduces its value exactly)
         float m_true = NEG_INF, m_ref = NEG_INF, l = 0.f, lr = 0.f;
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t mword = 0;
         unsigned int n_skip = 0;
 
-        for (int j = 0; j <= jmax[t]; j++) {
+        for (int j = 0; j <= jmaxt; j++) {
             if (!mbar_wait(&tl->s_full[t], j & 1, &tl->abort)) set_timeout(tl, p.status);
             tc_fence_after();
             uint32_t sr[128];
@@ -296,9 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 128; c++)
                     if (c > lim) s[c] = NEG_INF;
             }
-            float mx = NEG_INF;
+            // row max: four independent chains of 3-input max
+            float m0 = NEG_INF, m1 = NEG_INF, m2 = NEG_INF, m3 = NEG_INF;
 #pragma unroll
-            for (int c = 0; c < 128; c++) mx = fmaxf(mx, s[c]);
+            for (int c = 0; c < 128; c += 8) {
+                m0 = fmax3(m0, s[c], s[c + 1]);
+                m1 = fmax3(m1, s[c + 2], s[c + 3]);
+                m2 = fmax3(m2, s[c + 4], s[c + 5]);
+                m3 = fmax3(m3, s[c + 6], s[c + 7]);
+            }
+            const float mx = fmax3(m0, m1, fmaxf(m2, m3));
             const float mt = mx * p.scale_log2;  // -inf stays -inf (scale > 0)
             const float mn = fmaxf(m_true, mt);
             const bool vote = (mt == NEG_INF) || (mt - mn < p.thr_log2);
@@ -321,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mword |= 1u << (j & 31);
             }
             if (row == 0) {
-                if (p.skip_mask && ((j & 31) == 31 || j == jmax[t]))
+                if (p.skip_mask && ((j & 31) == 31 || j == jmaxt))
                     p.skip_mask[tile_idx * p.words + (j >> 5)] = mword;
                 tl->dec[t] = skip ? 0 : 1;
             }
@@ -334,57 +345,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_true = mn;
             // conditional rescale: only when the exp reference lags the true max by > 2^8
             const bool need = mn - m_ref > kRescaleThreshold;
-            if (__any_sync(0xffffffffu, need)) {
+            const bool warp_need = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (warp_need) {
                 const float m_new = mn;
-                const float alpha = (m_ref == NEG_INF || m_new == NEG_INF) ? (m_new == NEG_INF ? 1.f : 0.f)
-                                                                           : ex2(m_ref - m_new);
-                if (n_kept > 0) {
-                    if (!mbar_wait(&tl->o_done[t], (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
-                    tc_fence_after();
-                    uint32_t orr[32];
-#pragma unroll
-                    for (int c = 0; c < 4; c++) {
-                        tmem_ld32(o_addr + c * 32, orr);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; i++) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-                        tmem_st32(o_addr + c * 32, orr);
-                    }
-                }
+                alpha = (m_ref == NEG_INF || m_new == NEG_INF) ? (m_new == NEG_INF ? 1.f : 0.f) : ex2(m_ref - m_new);
                 l *= alpha;
                 lr *= alpha;
                 if (m_new != NEG_INF) m_ref = m_new;
             }
             const float mref = m_ref == NEG_INF ? 0.f : m_ref;
-            uint32_t pk[64];
-            float rs = 0.f, rr = 0.f;
+            float rs0 = 0.f, rs1 = 0.f, rr0 = 0.f, rr1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < 64; c++) {
-                const float p0 = ex2(fmaf(s[2 * c], p.scale_log2, -mref));
-                const float p1 = ex2(fmaf(s[2 * c + 1], p.scale_log2, -mref));
-                pk[c] = pack_bf16x2(p0, p1);
-                rs += p0 + p1;
-                rr += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+            for (int h = 0; h < 4; h++) {  // P in four chunks of 32 keys (16 packed columns)
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; c++) {
+                    const float p0 = ex2(fmaf(s[h * 32 + 2 * c], p.scale_log2, -mref));
+                    const float p1 = ex2(fmaf(s[h * 32 + 2 * c + 1], p.scale_log2, -mref));
+                    pk[c] = pack_bf16x2(p0, p1);
+                    if (c & 1) {
+                        rs1 += p0 + p1;
+                        rr1 += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+                    } else {
+                        rs0 += p0 + p1;
+                        rr0 += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+                    }
+                }
+                tmem_st16(s_addr + h * 16, pk);
             }
-            l += rs;
-            lr += rr;
-            tmem_st32(s_addr, pk);
-            tmem_st32(s_addr + 32, pk + 32);
+            l += rs0 + rs1;
+            lr += rr0 + rr1;
+            // O rescale after P is out of registers; P.V(j) is issued only after p_full
+            if (warp_need && n_kept > 0) {
+                if (!mbar_wait(&tl->o_done[t], (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    uint32_t orr[32];
+                    tmem_ld32(o_addr + c * 32, orr);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i++) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+                    tmem_st32(o_addr + c * 32, orr);
+                }
+            }
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(&tl->p_full[t]);
             n_kept++;
         }
-        if (jmax[t] >= 0) {
+        if (jmaxt >= 0) {
             if (row == 0 && p.skip_mask) {
-                for (int w = (jmax[t] >> 5) + 1; w < p.words; w++) p.skip_mask[tile_idx * p.words + w] = 0u;
+                for (int w = (jmaxt >> 5) + 1; w < p.words; w++) p.skip_mask[tile_idx * p.words + w] = 0u;
             }
             if (CALIB && row == 0 && p.gaps) {
-                for (int j = jmax[t] + 1; j < p.nb; j++) p.gaps[tile_idx * p.nb + j] = CUDART_NAN_F;
+                for (int j = jmaxt + 1; j < p.nb; j++) p.gaps[tile_idx * p.nb + j] = CUDART_NAN_F;
             }
             if (row == 0 && p.skip_count && n_skip) atomicAdd(p.skip_count, (unsigned long long)n_skip);
         }
-        if (!CALIB && jmax[t] >= 0) {
+        if (!CALIB && jmaxt >= 0) {
             // epilogue: O / l -> bf16, lse = (M_ref + log2 l) * ln 2
             if (!mbar_wait(&tl->o_done[t], (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
             tc_fence_after();

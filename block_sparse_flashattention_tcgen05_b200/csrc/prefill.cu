@@ -4,13 +4,14 @@
 // One CTA handles two 128-row query tiles (A, B) of one (sequence, query
 // head) that share every K/V block it loads.  d = dv = 128, KV blocks of 128.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3  softmax/decision warpgroup for tile A (thread i owns row i,
 //              i.e. TMEM lane i), warps 4-7 the same for tile B;
-//   warp 8     TMA producer: Q_A and Q_B once, then K_j and V_j into 2-stage
-//              rings (V is loaded for every block, as the prefill design of
-//              the pages keeps V prefetch regular);
-//   warp 9     allocates TMEM and issues every tcgen05.mma from one thread.
+//   warp 8     TMA producer: Q_A and Q_B once, then K_j into a 3-stage ring;
+//   warp 9     allocates TMEM and issues every tcgen05.mma from one thread;
+//   warp 10    TMA producer for V_j (2-stage ring; V is loaded for every
+//              block, as the prefill design of the pages keeps V prefetch
+//              regular), separate so the K stream never waits on a V slot.
 //
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
 // O_B [384,512); P_t (bf16, 64 columns) overwrites the first half of S_t.
@@ -39,11 +40,13 @@
 namespace blasst {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;   // Q and K
 constexpr int kMmaWarp = 9;
-constexpr int kStages = 2;
+constexpr int kVProducerWarp = 10;  // V
+constexpr int kStagesK = 3;
+constexpr int kStagesV = 2;
 constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
 constexpr int kBoxBytes = kTileBytes / 2;  // 128 rows x 64 bf16 (one swizzle box)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -51,8 +54,8 @@ constexpr int kStatusTimeout = 1;
 
 struct PrefillSmemTail {
     uint64_t q_full;
-    uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t v_full[kStages], v_empty[kStages];
+    uint64_t k_full[kStagesK], k_empty[kStagesK];
+    uint64_t v_full[kStagesV], v_empty[kStagesV];
     uint64_t s_full[2], p_full[2], o_done[2];
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -63,8 +66,8 @@ struct PrefillSmemTail {
 
 template <bool CALIB>
 constexpr int prefill_smem_bytes() {
-    return 2 * kTileBytes + kStages * kTileBytes + (CALIB ? 0 : kStages * kTileBytes) + (int)sizeof(PrefillSmemTail) +
-           1024;
+    return 2 * kTileBytes + kStagesK * kTileBytes + (CALIB ? 0 : kStagesV * kTileBytes) +
+           (int)sizeof(PrefillSmemTail) + 1024;
 }
 
 __device__ __forceinline__ void set_timeout(PrefillSmemTail *t, unsigned int *status) {
@@ -87,8 +90,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sq = smem;                                  // Q_A, Q_B
     uint8_t *sk = smem + 2 * kTileBytes;                 // K ring
-    uint8_t *sv = sk + kStages * kTileBytes;             // V ring
-    PrefillSmemTail *tl = reinterpret_cast<PrefillSmemTail *>(sv + (CALIB ? 0 : kStages * kTileBytes));
+    uint8_t *sv = sk + kStagesK * kTileBytes;            // V ring
+    PrefillSmemTail *tl = reinterpret_cast<PrefillSmemTail *>(sv + (CALIB ? 0 : kStagesV * kTileBytes));
 
     // longest rows first: blockIdx.x walks pairs of query tiles from the end
     const int n_pairs = (p.n_qtiles + 1) / 2;
@@ -103,15 +106,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&tl->q_full, 1);
-        for (int i = 0; i < kStages; i++) {
+        for (int i = 0; i < kStagesK; i++) {
             mbar_init(&tl->k_full[i], 1);
             mbar_init(&tl->k_empty[i], 1);
+        }
+        for (int i = 0; i < kStagesV; i++) {
             mbar_init(&tl->v_full[i], 1);
             mbar_init(&tl->v_empty[i], 1);
         }
         for (int t = 0; t < 2; t++) {
             mbar_init(&tl->s_full[t], 1);
-            mbar_init(&tl->p_full[t], kSoftmaxThreads);
+            mbar_init(&tl->p_full[t], kSoftmaxThreads / 32);
             mbar_init(&tl->o_done[t], 1);
         }
         mbar_init(&tl->mma_done, 1);
@@ -128,11 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = tl->tmem_base;
 
     if (warp == kProducerWarp) {
-        // ------------------------------------------------------------ TMA producer
+        // --------------------------------------------------------- TMA producer: Q, K
         if (lane == 0) {
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
-            if (!CALIB) tma_prefetch_desc(&tmap_v);
             const int qrow = b * p.Hq + hq;
             const int nq = jmax[1] >= 0 ? 2 : 1;
             mbar_arrive_expect_tx(&tl->q_full, nq * kTileBytes);
@@ -141,31 +145,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(sq + t * kTileBytes + kBoxBytes, &tmap_q, &tl->q_full, 64, q0[t], qrow);
             }
             const int kvrow = b * p.Hkv + hkv;
+            int issued = 0;
             for (int j = 0; j <= jmax_all && !tl->abort; j++) {
-                const int st = j % kStages;
-                const uint32_t par = ((j / kStages) & 1) ^ 1;
-                if (j >= kStages && !mbar_wait(&tl->k_empty[st], par, &tl->abort)) {
+                const int st = j % kStagesK;
+                if (j >= kStagesK && !mbar_wait(&tl->k_empty[st], ((j / kStagesK) & 1) ^ 1, &tl->abort)) {
                     set_timeout(tl, p.status);
                     break;
                 }
                 mbar_arrive_expect_tx(&tl->k_full[st], kTileBytes);
                 tma_load_3d(sk + st * kTileBytes, &tmap_k, &tl->k_full[st], 0, j * 128, kvrow);
                 tma_load_3d(sk + st * kTileBytes + kBoxBytes, &tmap_k, &tl->k_full[st], 64, j * 128, kvrow);
-                if (!CALIB) {
-                    if (j >= kStages && !mbar_wait(&tl->v_empty[st], par, &tl->abort)) {
-                        set_timeout(tl, p.status);
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&tl->v_full[st], kTileBytes);
-                    tma_load_3d(sv + st * kTileBytes, &tmap_v, &tl->v_full[st], 0, j * 128, kvrow);
-                    tma_load_3d(sv + st * kTileBytes + kBoxBytes, &tmap_v, &tl->v_full[st], 64, j * 128, kvrow);
-                }
+                issued++;
             }
             if (tl->abort) {  // let copies already issued land
-                for (int j = max(0, jmax_all - kStages + 1); j <= jmax_all; j++) {
-                    mbar_wait(&tl->k_full[j % kStages], (j / kStages) & 1, nullptr);
-                    if (!CALIB) mbar_wait(&tl->v_full[j % kStages], (j / kStages) & 1, nullptr);
+                for (int j = max(0, issued - kStagesK); j < issued; j++)
+                    mbar_wait(&tl->k_full[j % kStagesK], (j / kStagesK) & 1, nullptr);
+            }
+        }
+    } else if (warp == kVProducerWarp) {
+        // ------------------------------------------------------------ TMA producer: V
+        if (!CALIB && lane == 0) {
+            tma_prefetch_desc(&tmap_v);
+            const int kvrow = b * p.Hkv + hkv;
+            int issued = 0;
+            for (int j = 0; j <= jmax_all && !tl->abort; j++) {
+                const int st = j % kStagesV;
+                if (j >= kStagesV && !mbar_wait(&tl->v_empty[st], ((j / kStagesV) & 1) ^ 1, &tl->abort)) {
+                    set_timeout(tl, p.status);
+                    break;
                 }
+                mbar_arrive_expect_tx(&tl->v_full[st], kTileBytes);
+                tma_load_3d(sv + st * kTileBytes, &tmap_v, &tl->v_full[st], 0, j * 128, kvrow);
+                tma_load_3d(sv + st * kTileBytes + kBoxBytes, &tmap_v, &tl->v_full[st], 64, j * 128, kvrow);
+                issued++;
+            }
+            if (tl->abort) {
+                for (int j = max(0, issued - kStagesV); j < issued; j++)
+                    mbar_wait(&tl->v_full[j % kStagesV], (j / kStagesV) & 1, nullptr);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -177,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = mbar_wait(&tl->q_full, 0, &tl->abort);
             auto issue_s = [&](int t, int j) {
                 const uint32_t qa = smem_addr(sq + t * kTileBytes);
-                const uint32_t ka = smem_addr(sk + (j % kStages) * kTileBytes);
+                const uint32_t ka = smem_addr(sk + (j % kStagesK) * kTileBytes);
                 const uint32_t s_col = tmem + (uint32_t)t * 128u;
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++) {
@@ -195,12 +211,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&tl->k_empty[0]);
             }
             for (int j = 0; j <= jmax_all && ok; j++) {
-                const int st = j % kStages;
+                const int st = j % kStagesV;
                 bool v_waited = false;
                 bool k_next_waited = false;
 #pragma unroll
                 for (int t = 0; t < 2; t++) {
-                    if (j > jmax[t]) continue;
+                    if (j > jmax[t] || !ok) continue;
                     if (!mbar_wait(&tl->p_full[t], j & 1, &tl->abort)) {
                         set_timeout(tl, p.status);
                         ok = false;
@@ -210,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool kept = !CALIB && tl->dec[t] != 0;
                     if (kept) {
                         if (!v_waited) {
-                            if (!mbar_wait(&tl->v_full[st], (j / kStages) & 1, &tl->abort)) {
+                            if (!mbar_wait(&tl->v_full[st], (j / kStagesV) & 1, &tl->abort)) {
                                 set_timeout(tl, p.status);
                                 ok = false;
                                 break;
@@ -220,29 +236,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t va = smem_addr(sv + st * kTileBytes);
                         const uint32_t s_col = tmem + (uint32_t)t * 128u;
                         const uint32_t o_col = tmem + 256u + (uint32_t)t * 128u;
+                        const uint32_t acc0 = n_pv[t] > 0 ? 1u : 0u;
 #pragma unroll
                         for (int kk = 0; kk < 8; kk++)
                             umma_ts(o_col, s_col + kk * 8, umma_desc_sw128(va + kk * 2048, kBoxBytes), idesc_pv,
-                                    (n_pv[t] > 0 || kk > 0) ? 1u : 0u);
+                                    (acc0 || kk > 0) ? 1u : 0u);
                         umma_commit(&tl->o_done[t]);
                         n_pv[t]++;
                     }
                     if (j + 1 <= jmax[t]) {
                         if (!k_next_waited) {
-                            if (!mbar_wait(&tl->k_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, &tl->abort)) {
+                            if (!mbar_wait(&tl->k_full[(j + 1) % kStagesK], ((j + 1) / kStagesK) & 1, &tl->abort)) {
                                 set_timeout(tl, p.status);
                                 ok = false;
                                 break;
                             }
                             k_next_waited = true;
                         }
-                        // S_t(j+1) overwrites the columns holding P_t(j): wait for P.V to finish
-                        if (kept && !mbar_wait(&tl->o_done[t], (n_pv[t] - 1) & 1, &tl->abort)) {
-                            set_timeout(tl, p.status);
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
+                        // S_t(j+1) overwrites the columns that hold P_t(j).  tcgen05.mma
+                        // operations issued by one thread execute in issue order, so the
+                        // P.V above has read P before this product writes there.
                         issue_s(t, j + 1);
                     }
                 }
@@ -250,13 +263,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!CALIB) {
                     // consume V_j's load even when every tile skipped the block, so the
                     // slot's barrier phase is complete before the producer refills it
-                    if (!v_waited && !mbar_wait(&tl->v_full[st], (j / kStages) & 1, &tl->abort)) {
+                    if (!v_waited && !mbar_wait(&tl->v_full[st], (j / kStagesV) & 1, &tl->abort)) {
                         set_timeout(tl, p.status);
                         break;
                     }
                     umma_commit(&tl->v_empty[st]);
                 }
-                if (k_next_waited) umma_commit(&tl->k_empty[(j + 1) % kStages]);
+                if (k_next_waited) umma_commit(&tl->k_empty[(j + 1) % kStagesK]);
             }
             // every MMA and commit of this thread has completed before TMEM is released
             umma_commit(&tl->mma_done);
@@ -327,21 +340,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 bar_sync(bar_id, kSoftmaxThreads);
             }
-            if (skip) {
-                n_skip++;
-                mword |= 1u << (j & 31);
-            }
-            if (row == 0) {
-                if (p.skip_mask && ((j & 31) == 31 || j == jmaxt))
-                    p.skip_mask[tile_idx * p.words + (j >> 5)] = mword;
-                tl->dec[t] = skip ? 0 : 1;
-            }
-            if ((j & 31) == 31) mword = 0;
+            if (row == 0) tl->dec[t] = skip ? 0 : 1;
             if (skip || CALIB) {
                 if (!skip) m_true = mn;
-                mbar_arrive(&tl->p_full[t]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tl->p_full[t]);
+                if (skip) {
+                    n_skip++;
+                    mword |= 1u << (j & 31);
+                }
+                if (row == 0 && p.skip_mask && ((j & 31) == 31 || j == jmaxt))
+                    p.skip_mask[tile_idx * p.words + (j >> 5)] = mword;
+                if ((j & 31) == 31) mword = 0;
                 continue;
             }
+            if (row == 0 && p.skip_mask && ((j & 31) == 31 || j == jmaxt))
+                p.skip_mask[tile_idx * p.words + (j >> 5)] = mword;
+            if ((j & 31) == 31) mword = 0;
             m_true = mn;
             // conditional rescale: only when the exp reference lags the true max by > 2^8
             const bool need = mn - m_ref > kRescaleThreshold;
@@ -355,27 +370,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (m_new != NEG_INF) m_ref = m_new;
             }
             const float mref = m_ref == NEG_INF ? 0.f : m_ref;
-            float rs0 = 0.f, rs1 = 0.f, rr0 = 0.f, rr1 = 0.f;
+            const uint64_t scl2 = f2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t neg2 = f2_pack(-mref, -mref);
+            uint64_t rs2a = 0, rs2b = 0, rr2a = 0, rr2b = 0;  // packed {lo, hi} partial sums (0 == +0.0f pair)
 #pragma unroll
             for (int h = 0; h < 4; h++) {  // P in four chunks of 32 keys (16 packed columns)
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 16; c++) {
-                    const float p0 = ex2(fmaf(s[h * 32 + 2 * c], p.scale_log2, -mref));
-                    const float p1 = ex2(fmaf(s[h * 32 + 2 * c + 1], p.scale_log2, -mref));
+                    const uint64_t y = f2_fma(f2_pack(s[h * 32 + 2 * c], s[h * 32 + 2 * c + 1]), scl2, neg2);
+                    float y0, y1;
+                    f2_unpack(y, y0, y1);
+                    const float p0 = ex2(y0), p1 = ex2(y1);
                     pk[c] = pack_bf16x2(p0, p1);
                     if (c & 1) {
-                        rs1 += p0 + p1;
-                        rr1 += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+                        rs2b = f2_add(rs2b, f2_pack(p0, p1));
+                        rr2b = f2_add(rr2b, bf16x2_widen(pk[c]));
                     } else {
-                        rs0 += p0 + p1;
-                        rr0 += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+                        rs2a = f2_add(rs2a, f2_pack(p0, p1));
+                        rr2a = f2_add(rr2a, bf16x2_widen(pk[c]));
                     }
                 }
                 tmem_st16(s_addr + h * 16, pk);
             }
-            l += rs0 + rs1;
-            lr += rr0 + rr1;
+            {
+                float a0, a1, b0, b1;
+                f2_unpack(f2_add(rs2a, rs2b), a0, a1);
+                f2_unpack(f2_add(rr2a, rr2b), b0, b1);
+                l += a0 + a1;
+                lr += b0 + b1;
+            }
             // O rescale after P is out of registers; P.V(j) is issued only after p_full
             if (warp_need && n_kept > 0) {
                 if (!mbar_wait(&tl->o_done[t], (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
@@ -392,7 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&tl->p_full[t]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->p_full[t]);
             n_kept++;
         }
         if (jmaxt >= 0) {

@@ -191,14 +191,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 128, 1);
             int n_pv[2] = {0, 0};
             bool ok = mbar_wait(&tl->q_full, 0, &tl->abort);
+            // descriptor low halves (start address | LBO); the high half is shared
+            constexpr uint32_t dhi = umma_desc_hi_sw128();
+            const uint32_t q_lo0 = umma_desc_lo(smem_addr(sq), 16);
+            const uint32_t k_lo0 = umma_desc_lo(smem_addr(sk), 16);
+            const uint32_t v_lo0 = umma_desc_lo(smem_addr(sv), kBoxBytes);
             auto issue_s = [&](int t, int j) {
-                const uint32_t qa = smem_addr(sq + t * kTileBytes);
-                const uint32_t ka = smem_addr(sk + (j % kStagesK) * kTileBytes);
+                const uint32_t qa = q_lo0 + (uint32_t)t * (kTileBytes >> 4);
+                const uint32_t ka = k_lo0 + (uint32_t)(j % kStagesK) * (kTileBytes >> 4);
                 const uint32_t s_col = tmem + (uint32_t)t * 128u;
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++) {
-                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    umma_ss(s_col, umma_desc_sw128(qa + off, 16), umma_desc_sw128(ka + off, 16), idesc_s, kk > 0);
+                    const uint32_t off = (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+                    umma_ss2(s_col, qa + off, ka + off, dhi, idesc_s, kk > 0);
                 }
                 umma_commit(&tl->s_full[t]);
             };
@@ -233,14 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             v_waited = true;
                         }
-                        const uint32_t va = smem_addr(sv + st * kTileBytes);
+                        const uint32_t va = v_lo0 + (uint32_t)st * (kTileBytes >> 4);
                         const uint32_t s_col = tmem + (uint32_t)t * 128u;
                         const uint32_t o_col = tmem + 256u + (uint32_t)t * 128u;
                         const uint32_t acc0 = n_pv[t] > 0 ? 1u : 0u;
 #pragma unroll
                         for (int kk = 0; kk < 8; kk++)
-                            umma_ts(o_col, s_col + kk * 8, umma_desc_sw128(va + kk * 2048, kBoxBytes), idesc_pv,
-                                    (acc0 || kk > 0) ? 1u : 0u);
+                            umma_ts2(o_col, s_col + kk * 8, va + kk * (2048 >> 4), dhi, idesc_pv,
+                                     (acc0 || kk > 0) ? 1u : 0u);
                         umma_commit(&tl->o_done[t]);
                         n_pv[t]++;
                     }

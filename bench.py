@@ -45,12 +45,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, Hq=32, Hkv=8, L=32768, d=128,
                causal=True, seed=2)
 DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk=32768, d=128, splits=16, seed=3)
+MLA = dict(workload="MLA decode, 128 heads, 576/512 latent, 32K cache, 2 splits", B=64, Hq=128, Lk=32768, splits=2,
+           seed=5)
 QUICK_PREFILL = dict(PREFILL, workload="prefill GQA 4K (quick)", L=4096)
 QUICK_DECODE = dict(DECODE, workload="decode GQA 4K cache (quick)", B=4, Lk=4096)
 # profiling size: inputs larger than L2 (126 MB) but a few GB at most on the device
 MEDIUM_PREFILL = dict(PREFILL, workload="prefill GQA 16K (profiling size)", L=16384)
 MEDIUM_DECODE = dict(DECODE, workload="decode GQA 32K cache, batch 8 (profiling size)", B=8)
-SIZES = {"full": (PREFILL, DECODE), "medium": (MEDIUM_PREFILL, MEDIUM_DECODE), "quick": (QUICK_PREFILL, QUICK_DECODE)}
+MEDIUM_MLA = dict(MLA, workload="MLA decode, batch 16 (profiling size)", B=16)
+QUICK_MLA = dict(MLA, workload="MLA decode (quick)", B=2, Lk=4096)
+SIZES = {"full": (PREFILL, DECODE, MLA), "medium": (MEDIUM_PREFILL, MEDIUM_DECODE, MEDIUM_MLA),
+         "quick": (QUICK_PREFILL, QUICK_DECODE, QUICK_MLA)}
 TARGETS = (0.0, 0.5, 0.75)
 
 
@@ -271,6 +276,57 @@ class Decode:
         hl.copy_(self.lse, non_blocking=True)
 
 
+class Mla:
+    """MLA decode: 576-column latent cache (V = first 512 columns), all heads in one tile."""
+
+    kind = "mla"
+    unit = "GB/s"
+    bound = "hbm"
+
+    def __init__(self, cfg, device):
+        import synth
+
+        self.cfg = cfg
+        self.device = device
+        c = cfg
+        self.inp = synth.planted_mla(c["B"], c["Hq"], c["Lk"], seed=c["seed"], reading="blk")
+        self.q, self.k = (to_dev(x, device) for x in (self.inp.q, self.inp.k))
+        self.v = self.k
+        import torch
+
+        import block_sparse_flashattention_tcgen05_b200 as bl
+
+        self.bl = bl
+        self.o = torch.empty((c["B"], c["Hq"], 1, 512), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((c["B"], c["Hq"], 1), dtype=torch.float32, device=device)
+        self.ws = torch.empty(bl.decode_workspace_bytes(c["B"], c["Hq"], 1, 512, c["splits"]), dtype=torch.uint8,
+                              device=device)
+        self.visited = bl.visited_pairs(c["B"], c["Hq"], 1, 1, c["Lk"], False, True)
+        self.launches = 2
+
+    def calibrate(self):
+        gaps, _, _ = self.bl.calibrate(self.q, self.k, scale=self.inp.scale, causal=False, mode="decode",
+                                       num_splits=self.cfg["splits"], dv=512)
+        return gaps.cpu().numpy()
+
+    def call(self, lam, stream=None):
+        return self.bl.decode(self.q, self.k, self.k, scale=self.inp.scale, lam=lam, num_splits=self.cfg["splits"],
+                              dv=512, o=self.o, lse=self.lse, skip_mask=False, skip_count=self.count,
+                              workspace=self.ws, stream=stream)
+
+    def work(self, skipped):
+        c = self.cfg
+        return c["B"] * c["Lk"] * 576 * 2 + self.inp.q.nbytes + self.o.numel() * 2 + self.lse.numel() * 4
+
+    def flops(self, skipped):
+        c = self.cfg
+        kept = self.visited - skipped
+        return 2 * c["Hq"] * 64 * 576 * self.visited + 2 * c["Hq"] * 64 * 512 * kept
+
+    def rate(self, work, ms):
+        return work / (ms * 1e-3) / 1e9
+
+
 def lambdas_for_targets(wl, gaps):
     out = {}
     for t in TARGETS:
@@ -461,6 +517,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-mla", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -482,7 +539,7 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     notes = []
 
-    pcfg, dcfg = SIZES[args.size]
+    pcfg, dcfg, mcfg = SIZES[args.size]
     headline_kind = args.workload
     wls = {}
     try:
@@ -498,6 +555,8 @@ def main():
         headline_kind = "decode"
     if headline_kind == "decode" or not args.no_sweep:
         wls["decode"] = Decode(dcfg, dev)
+    if not args.no_sweep and not args.no_mla:
+        wls["mla"] = Mla(mcfg, dev)
 
     lams = {k: lambdas_for_targets(w, w.calibrate()) for k, w in wls.items()}
 
@@ -548,6 +607,9 @@ def main():
                     "lambda": lam, "a=lambda*L": lam * (w.cfg.get("L") or w.cfg.get("Lk")),
                     "sparsity": sk / w.visited, "ms": med, "value": r, "unit": w.unit,
                     "frac_of_measured_peak": r / pk, "speedup_vs_lambda0": base / med}
+                if hasattr(w, "flops"):
+                    tf = w.flops(sk) / (med * 1e-3) / 1e12
+                    rows[f"{int(t * 100)}%"].update(tflops=tf, tensor_frac_of_measured_peak=tf / peaks["bf16_tflops"])
             sweep[kind] = rows
 
     # ---- end to end through the public API with host buffers

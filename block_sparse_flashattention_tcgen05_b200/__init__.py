@@ -167,10 +167,13 @@ def prefill(q, k, v, *, scale, lam=0.0, causal=True, o=None, lse=None, skip_mask
     return o, lse, m, c
 
 
-def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=None, skip_mask=True,
-           skip_count=True, workspace=None, status_word=None, stream=None):
-    """Split-KV decode with block skipping.  q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA.
+def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o=None, lse=None,
+           skip_mask=True, skip_count=True, workspace=None, status_word=None, stream=None):
+    """Split-KV decode with block skipping.
 
+    GQA/MQA: q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA (16 splits by default).
+    MLA: q [B,Hq,Lq,576], k [B,1,Lk,576], v = the same tensor as k, dv = 512 (V is
+    the first 512 columns of each cache row; 2 splits by default).
     Returns (o, lse, skip_mask [B*Hkv, W] int32 or None, skip_count [1] int64 or None).
     ``workspace``: optional uint8 CUDA tensor of at least decode_workspace_bytes() bytes.
     """
@@ -178,13 +181,14 @@ def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=
 
     _dev_tensor(q, "q"), _dev_tensor(k, "k"), _dev_tensor(v, "v")
     B, Hq, Lq, d = q.shape
-    _, Hkv, Lk, _ = k.shape
-    dv = v.shape[-1]
+    _, Hkv, Lk, krs = k.shape
+    vrs = v.shape[-1]
+    dv = vrs if dv is None else dv
     if o is None:
         o = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    opts = Opts(num_splits=num_splits, dv=dv,
+    opts = Opts(num_splits=num_splits or 0, dv=dv, k_row_stride=krs, v_row_stride=vrs,
                 status_word=None if status_word is None else status_word.data_ptr())
     if workspace is not None:
         opts.workspace = workspace.data_ptr()
@@ -223,7 +227,7 @@ def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=No
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
-def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=16, skip_mask=True,
+def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=None, dv=None, skip_mask=True,
               skip_count=True, stream=None):
     """Decision-only pass.  Returns (gaps [tiles, nb] fp32, skip_mask, skip_count)."""
     import torch
@@ -242,7 +246,7 @@ def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=1
     else:
         raise ValueError(mode)
     gaps = torch.empty((tiles, nb), dtype=torch.float32, device=q.device)
-    opts = Opts(mode=m, num_splits=num_splits, gaps_out=gaps.data_ptr())
+    opts = Opts(mode=m, num_splits=num_splits or 0, gaps_out=gaps.data_ptr(), dv=dv or 0)
     mk, c = _attn("blasst_calibrate", q, k, None, scale=scale, lam=lam, causal=causal, o=None, lse=None,
                   want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=tiles,
                   n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=d)

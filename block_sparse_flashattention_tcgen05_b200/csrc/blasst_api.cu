@@ -112,6 +112,81 @@ float log2_threshold(float lambda) {
 
 const double kLog2e = 1.4426950408889634;
 
+// ---------------------------------------------------------------------- MLA
+blasst_status run_mla(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                      int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
+                      unsigned long long *skip_count, void *stream, const blasst_opts &op, const Common &c,
+                      bool calib) {
+    // one latent KV head; V = the first 512 columns of the same cache rows
+    if (Hkv != 1 || c.dv != 512 || c.krs != d) return BLASST_ERR_UNSUPPORTED;
+    if (!calib && (v != k || c.vrs != c.krs)) return BLASST_ERR_UNSUPPORTED;
+    const long long R = (long long)Hq * Lq;
+    if (R > 128) return BLASST_ERR_UNSUPPORTED;
+    const int S = op.num_splits ? op.num_splits : 2;
+    if (S < 1 || S > 65535 || B > 65535) return BLASST_ERR_INVALID;
+    const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
+    const int per_split = (nb + S - 1) / S;
+    const int words = (nb + 31) / 32;
+    const size_t rows = (size_t)B * Hq * Lq;
+    const size_t need = blasst_decode_workspace_bytes(B, Hq, Lq, c.dv, S);
+    void *ws = op.workspace;
+    if (!calib && ws && op.workspace_bytes < need) return BLASST_ERR_WORKSPACE;
+    cudaStream_t sm = reinterpret_cast<cudaStream_t>(stream);
+
+    CUtensorMap tq, tk;
+    blasst_status st = make_tmap(&tq, q, d, R, B, d, 64, 128);
+    if (st != BLASST_OK) return st;
+    st = make_tmap(&tk, k, d, Lk, B, c.krs, 64, kDecodeBlockN);
+    if (st != BLASST_OK) return st;
+    bool own_ws = false;
+    cudaError_t e;
+    if (!calib && !ws) {
+        e = cudaMallocAsync(&ws, need, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        own_ws = true;
+    }
+    if (skip_mask) {
+        e = cudaMemsetAsync(skip_mask, 0, (size_t)B * words * sizeof(uint32_t), sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_mask)");
+    }
+    if (skip_count) {
+        e = cudaMemsetAsync(skip_count, 0, sizeof(unsigned long long), sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_count)");
+    }
+    MlaParams p;
+    std::memset(&p, 0, sizeof p);
+    p.part_o = calib ? nullptr : static_cast<float *>(ws);
+    p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));
+    p.skip_mask = skip_mask;
+    p.skip_count = skip_count;
+    p.gaps = op.gaps_out;
+    p.status = op.status_word;
+    p.B = B; p.Hq = Hq; p.Lq = Lq; p.Lk = Lk; p.R = (int)R;
+    p.nb = nb; p.num_splits = S; p.per_split = per_split; p.words = words;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = (float)(scale * kLog2e);
+    p.thr_log2 = log2_threshold(lambda);
+    e = launch_mla(p, tq, tk, calib, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "MLA split kernel");
+    if (!calib) {
+        CombineParams cp;
+        cp.part_o = p.part_o;
+        cp.part_lse = p.part_lse;
+        cp.o = static_cast<uint16_t *>(o);
+        cp.lse = lse;
+        cp.rows = (int)rows;
+        cp.num_splits = S;
+        cp.dv = c.dv;
+        e = launch_combine(cp, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel");
+    }
+    if (own_ws) {
+        e = cudaFreeAsync(ws, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    }
+    return BLASST_OK;
+}
+
 // ------------------------------------------------------------------- decode
 blasst_status run_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                          int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
@@ -127,6 +202,8 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         return BLASST_ERR_INVALID;
     }
     if (op.block_n != 0 && op.block_n != kDecodeBlockN) return BLASST_ERR_UNSUPPORTED;
+    if (d == 576) return run_mla(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count,
+                                 stream, op, c, calib);
     if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
     const int G = Hq / Hkv;
     const long long R = (long long)G * Lq;

@@ -53,12 +53,30 @@ struct PrefillParams {
     float thr_log2;
 };
 
+// One MLA decode (or MLA-shaped calibration) call: a single latent KV head of
+// 576 columns, V = its first 512 columns.
+struct MlaParams {
+    float *part_o;                  // [B*Hq*Lq, S, 512] fp32 split outputs (normalised)
+    float *part_lse;                // [B*Hq*Lq, S]
+    uint32_t *skip_mask;            // [B, 1, 1, W] or null
+    unsigned long long *skip_count; // or null
+    float *gaps;                    // [B, nb] or null
+    unsigned int *status;           // or null
+    int B, Hq, Lq, Lk, R;           // R = Hq * Lq <= 128
+    int nb, num_splits, per_split, words;
+    int causal;
+    float scale_log2;
+    float thr_log2;
+};
+
 // Records the text returned by blasst_last_error() for this thread.
 void set_last_error(const char *msg);
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
                           int nt, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t stream);
+cudaError_t launch_mla(const MlaParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k, bool calib,
+                       cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
                            const CUtensorMap &tmap_v, bool calib, cudaStream_t stream);
 

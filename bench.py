@@ -47,6 +47,7 @@ PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, H
 DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk=32768, d=128, splits=16, seed=3)
 MLA = dict(workload="MLA decode, 128 heads, 576/512 latent, 32K cache, 2 splits", B=64, Hq=128, Lk=32768, splits=2,
            seed=5)
+PREFILL_64K = dict(PREFILL, workload="prefill GQA 64K (Qwen3-8B-like attention shape)", L=65536, seed=4)
 QUICK_PREFILL = dict(PREFILL, workload="prefill GQA 4K (quick)", L=4096)
 QUICK_DECODE = dict(DECODE, workload="decode GQA 4K cache (quick)", B=4, Lk=4096)
 # profiling size: inputs larger than L2 (126 MB) but a few GB at most on the device
@@ -388,6 +389,64 @@ def e2e_measure(wl, lam, steps, warmup):
     return ms, skipped, hb, db
 
 
+# ------------------------------------------------------------- calibration sweep
+def calibration_sweep(device, lengths, targets=(0.3, 0.4, 0.5, 0.6, 0.7, 0.8), B=1, Hq=32, Hkv=8, seed=7):
+    """Fit lambda*L = alpha*exp(beta*s) across context lengths (one decision-only pass per L).
+
+    For each L: gaps from blasst_calibrate; per target s the lambda reaching s (gap quantile), a = lambda*L.
+    Fit over all reachable (L, s) points with blasst_calibrate_fit, then report, per L and s, the sparsity
+    reached by the fitted lambda = a(s)/L, and by one fixed lambda (the one giving 50% at the middle L)."""
+    import numpy as np
+    import torch
+
+    import block_sparse_flashattention_tcgen05_b200 as bl
+    import synth
+
+    per_L = {}
+    pts_L, pts_lam, pts_s = [], [], []
+    for L in lengths:
+        inp = synth.planted_prefill(B, Hq, Hkv, L, 128, seed=seed, reading="blk")
+        q, k = to_dev(inp.q, device), to_dev(inp.k, device)
+        t0 = time.time()
+        gaps, _, _ = bl.calibrate(q, k, scale=inp.scale, causal=True, mode="prefill")
+        torch.cuda.synchronize()
+        g = gaps.cpu().numpy()
+        per_L[L] = dict(gaps=g, visited=int(np.count_nonzero(~np.isnan(g))), calib_s=time.time() - t0)
+        for t in targets:
+            lam, ach = bl.calibrate_threshold(g, t)
+            if lam > 0 and abs(ach - t) < 0.01:
+                pts_L.append(L)
+                pts_lam.append(lam)
+                pts_s.append(ach)
+        del q, k, gaps
+    alpha, beta = bl.calibrate_fit(pts_L, pts_lam, pts_s)
+
+    def sparsity_at(g, lam):
+        fin = g[~np.isnan(g)]
+        return float(np.count_nonzero(fin < math.log(lam))) / fin.size if lam > 0 else 0.0
+
+    mid = lengths[len(lengths) // 2]
+    lam_fixed, _ = bl.calibrate_threshold(per_L[mid]["gaps"], 0.5)
+    rows = []
+    errs = []
+    for L in lengths:
+        g = per_L[L]["gaps"]
+        for t in targets:
+            lam_fit = min(alpha * math.exp(beta * t) / L, 1.0 - 1e-7)
+            sp = sparsity_at(g, lam_fit)
+            errs.append(abs(sp - t))
+            rows.append({"L": L, "target": t, "a_fit": alpha * math.exp(beta * t), "lambda_fit": lam_fit,
+                         "achieved": sp, "abs_error": abs(sp - t)})
+    fixed = {str(L): sparsity_at(per_L[L]["gaps"], lam_fixed) for L in lengths}
+    cal50 = {str(L): sparsity_at(per_L[L]["gaps"], min(alpha * math.exp(beta * 0.5) / L, 1 - 1e-7))
+             for L in lengths}
+    return {"alpha": alpha, "beta": beta, "points": len(pts_s), "mean_abs_sparsity_error": float(np.mean(errs)),
+            "max_abs_sparsity_error": float(np.max(errs)), "per_point": rows,
+            "fixed_lambda": {"lambda": lam_fixed, "sparsity_by_L": fixed},
+            "calibrated_50pct_sparsity_by_L": cal50,
+            "workload": f"prefill GQA B={B} Hq={Hq} Hkv={Hkv} d=128 causal, 'blk' inputs seed {seed}"}
+
+
 # ------------------------------------------------------------------ CPU baseline
 def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
     """Time the fp64 oracle (as it stands) on a bounded sample of query tiles.
@@ -518,6 +577,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mla", action="store_true")
+    ap.add_argument("--no-64k", action="store_true")
+    ap.add_argument("--calibration", action="store_true",
+                    help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -557,6 +619,8 @@ def main():
         wls["decode"] = Decode(dcfg, dev)
     if not args.no_sweep and not args.no_mla:
         wls["mla"] = Mla(mcfg, dev)
+    if not args.no_sweep and args.size == "full" and "prefill" in wls and not args.no_64k:
+        wls["prefill_64k"] = Prefill(PREFILL_64K, dev)
 
     lams = {k: lambdas_for_targets(w, w.calibrate()) for k, w in wls.items()}
 
@@ -612,6 +676,12 @@ def main():
                     rows[f"{int(t * 100)}%"].update(tflops=tf, tensor_frac_of_measured_peak=tf / peaks["bf16_tflops"])
             sweep[kind] = rows
 
+    # ---- calibration fit across context lengths (prefill-shaped decision pass)
+    calib = None
+    if args.calibration and "prefill" in wls:
+        lengths = (8192, 16384, 32768, 65536) if args.size == "full" else (2048, 4096, 8192)
+        calib = calibration_sweep(dev, lengths)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -636,7 +706,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": t_max * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfgd,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": wl.launches * args.steps,
-        "clocks": clocks, "sweep": sweep, "notes": notes,
+        "clocks": clocks, "sweep": sweep, "calibration": calib, "notes": notes,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -185,3 +185,12 @@ def test_prefill_full_size_sampled(bl, lam):
     nq = 256
     tiles = np.sort(np.concatenate([rng.choice(32 * nq, 6, replace=False), [nq - 1, 31 * nq + nq - 1]]))
     check_prefill(bl, inp, lam, True, tiles=tiles)
+
+
+@pytest.mark.slow
+def test_prefill_64k_sampled(bl):
+    # the long-context launch: B=1, Hq=32, Hkv=8, L=65536, causal; oracle on sampled tiles
+    inp = planted_prefill(1, 32, 8, 65536, 128, seed=4, reading="blk")
+    nq = 512
+    tiles = [nq - 1, 5 * nq + 200, 17 * nq + 3, 31 * nq + nq - 1]
+    check_prefill(bl, inp, 3e-3, True, tiles=tiles)

@@ -71,15 +71,28 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def load_profile_traffic(kernel_key):
-    """DRAM bytes per launch from a committed ncu summary, if it is current."""
+def load_profile_counters(kernel_key):
+    """ncu counters of the benchmarked launch from the committed summary
+    (profiles/traffic.json): {"dram_bytes_per_launch", "tensor_pipe_active_pct",
+    ...}, or {} when none were taken for the current kernel build."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        return d.get(kernel_key)
+        return d.get(kernel_key) or {}
     except Exception:
-        return None
+        return {}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 class ClockSampler:
@@ -502,6 +515,48 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
                 seconds=dt)
 
 
+def oracle_mha1024(lam_a=32.0, budget_s=3.0):
+    """The oracle on the whole 1024-token MHA prefill (planted generator,
+    lambda = a/L), repeated for about budget_s; effective TFLOP/s."""
+    import oracle
+    import synth
+
+    L = 1024
+    inp = synth.planted_prefill(1, 1, 1, L, 128, seed=1, reading="lit", boost=False)
+    n, t0 = 0, time.time()
+    while True:
+        r = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=lam_a / L, causal=True)
+        n += 1
+        if time.time() - t0 >= budget_s:
+            break
+    dt = time.time() - t0
+    work = FLOP_PER_PAIR * (2 * r["n_visited"] - r["n_skipped"]) * n / 1e12
+    return {"value": work / dt, "unit": "TFLOP/s", "sample": f"whole 1024-token MHA prefill, lambda={lam_a:g}/L, "
+            f"{n} runs in {dt:.1f} s"}
+
+
+def single_core_oracle(dcfg):
+    """The oracle on one host core (child process, OMP_NUM_THREADS=1): the
+    1024-token MHA prefill in full and a sample of the GQA decode workload."""
+    import subprocess
+
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    cmd = [sys.executable, os.path.abspath(__file__), "--single-core-oracle", json.dumps(dcfg)]
+    try:
+        out = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=120, check=True).stdout
+        return json.loads(out.strip().splitlines()[-1])
+    except Exception as e:  # reported, never fatal to the GPU measurement
+        return {"error": f"{type(e).__name__}: {e}"[:200]}
+
+
+def _single_core_main(dcfg_json):
+    dcfg = json.loads(dcfg_json)
+    res = {"threads": int(os.environ.get("OMP_NUM_THREADS", "0")), "mha_prefill_1024": oracle_mha1024()}
+    d = oracle_sample("decode", dcfg, budget_s=4.0)
+    res["decode"] = {k: d[k] for k in ("value", "unit", "sample")}
+    print(json.dumps(res), flush=True)
+
+
 # -------------------------------------------------------------------------- main
 def dist_setup(args):
     import torch
@@ -565,6 +620,9 @@ def run_reference(args, world, rank):
 
 
 def main():
+    if len(sys.argv) == 3 and sys.argv[1] == "--single-core-oracle":
+        _single_core_main(sys.argv[2])
+        return
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -647,11 +705,18 @@ def main():
     if wl.bound == "tensor":
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peak_src} bf16 burst", "traffic": load_profile_traffic("prefill")}
+                "peak_source": f"{peak_src} bf16 burst"}
     else:
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "peak_source": f"{peak_src} copy bandwidth", "traffic": load_profile_traffic("decode")}
+                "peak_source": f"{peak_src} copy bandwidth"}
+
+    prof = load_profile_counters("prefill" if wl.bound == "tensor" else "decode")
+    roof["traffic"] = prof.get("dram_bytes_per_launch")
+    if wl.bound == "tensor":
+        roof["tensor_pipe_active_pct_ncu"] = prof.get("tensor_pipe_active_pct")
+    if prof:
+        roof["ncu_source"] = prof.get("source")
 
     # ---- sweep: 0/50/75% on both workloads, speedup over lambda = 0
     sweep = {}
@@ -671,6 +736,9 @@ def main():
                     "lambda": lam, "a=lambda*L": lam * (w.cfg.get("L") or w.cfg.get("Lk")),
                     "sparsity": sk / w.visited, "ms": med, "value": r, "unit": w.unit,
                     "frac_of_measured_peak": r / pk, "speedup_vs_lambda0": base / med}
+                if w.kind == "prefill":
+                    # each skipped pair omits its 128 x 128 exponentials: the skipped-exp share is the sparsity
+                    rows[f"{int(t * 100)}%"]["exp_skipped_fraction"] = sk / w.visited
                 if hasattr(w, "flops"):
                     tf = w.flops(sk) / (med * 1e-3) / 1e12
                     rows[f"{int(t * 100)}%"].update(tflops=tf, tensor_frac_of_measured_peak=tf / peaks["bf16_tflops"])
@@ -694,6 +762,10 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample(headline_kind, wl.cfg, budget_s=float(os.environ.get("BLASST_CPU_SECONDS", "12")))
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        cpu["cpu_model"] = cpu_model()
+        cpu["nproc"] = os.cpu_count()
+        # per-tile work is the same at any batch: a batch of 4 keeps the generator cheap
+        cpu["single_core"] = single_core_oracle(dict(dcfg, B=min(4, dcfg["B"])))
 
     cfgd = {"workload": wl.cfg["workload"], "lambda": lam75, "target_sparsity": 0.75, "achieved_sparsity":
             skipped / wl.visited, "visited_pairs": wl.visited, "reading": "blk",

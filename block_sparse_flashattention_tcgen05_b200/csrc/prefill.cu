@@ -57,9 +57,11 @@ struct PrefillSmemTail {
     uint64_t k_full[kStagesK], k_empty[kStagesK];
     uint64_t v_full[kStagesV], v_empty[kStagesV];
     uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t vote_bar[2];  // one arrival per softmax warp and block (blocks j >= 1)
     uint64_t mma_done;
     uint32_t tmem_base;
     int dec[2];
+    uint32_t votes[2][2];  // [tile][block parity]: byte w = warp w's rows all allow the skip
     int abort;
     float gred[2][4];
 };
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tl->s_full[t], 1);
             mbar_init(&tl->p_full[t], kSoftmaxThreads / 32);
             mbar_init(&tl->o_done[t], 1);
+            mbar_init(&tl->vote_bar[t], kSoftmaxThreads / 32);
         }
         mbar_init(&tl->mma_done, 1);
         tl->abort = 0;
@@ -331,8 +334,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mt = mx * p.scale_log2;  // -inf stays -inf (scale > 0)
             const float mn = fmaxf(m_true, mt);
             const bool vote = (mt == NEG_INF) || (mt - mn < p.thr_log2);
-            const bool all = bar_and(bar_id, kSoftmaxThreads, vote);
-            const bool skip = all && j > 0;
+            // Tile-wide AND in two levels.  A warp with a row that forbids the skip
+            // knows the block is kept and goes on at once; only a warp whose rows all
+            // allow it waits for the other three warps' votes.  The first block is
+            // always kept and takes no vote.  (A warp reaches block j+1 only after all
+            // four warps published block j, so one barrier phase per block suffices.)
+            bool skip = false;
+            if (j > 0) {
+                const bool wvote = __all_sync(0xffffffffu, vote);
+                uint8_t *vb = reinterpret_cast<uint8_t *>(&tl->votes[t][j & 1]);
+                if (lane == 0) {
+                    vb[wq] = wvote ? 1 : 0;
+                    mbar_arrive(&tl->vote_bar[t]);  // release: the vote byte is visible first
+                }
+                if (wvote) {
+                    if (mbar_wait(&tl->vote_bar[t], (j - 1) & 1, &tl->abort))
+                        skip = *reinterpret_cast<volatile uint32_t *>(vb) == 0x01010101u;
+                    else
+                        set_timeout(tl, p.status);
+                }
+            }
             if (CALIB && p.gaps) {
                 float g = mt == NEG_INF ? NEG_INF : mt - mn;
 #pragma unroll

@@ -155,6 +155,7 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
     }
     MlaParams p;
     std::memset(&p, 0, sizeof p);
+    p.q = static_cast<const uint16_t *>(q);
     p.part_o = calib ? nullptr : static_cast<float *>(ws);
     p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));
     p.skip_mask = skip_mask;
@@ -253,6 +254,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
 
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
+    p.q = static_cast<const uint16_t *>(q);
     p.q = static_cast<const uint16_t *>(q);
     p.part_o = calib ? nullptr : static_cast<float *>(ws);
     p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));

@@ -56,6 +56,7 @@ struct PrefillParams {
 // One MLA decode (or MLA-shaped calibration) call: a single latent KV head of
 // 576 columns, V = its first 512 columns.
 struct MlaParams {
+    const uint16_t *q;              // [B, Hq*Lq, 576] bf16 queries (dense rows)
     float *part_o;                  // [B*Hq*Lq, S, 512] fp32 split outputs (normalised)
     float *part_lse;                // [B*Hq*Lq, S]
     uint32_t *skip_mask;            // [B, 1, 1, W] or null

@@ -99,8 +99,9 @@ class ClockSampler:
     """SM clock and clock-event (throttle) reasons, polled through NVML every
     few milliseconds while the timed region runs (read-only queries)."""
 
-    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
-               0x80: "hw_power_brake_slowdown"}
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, device_index):
         self.samples = []
@@ -157,12 +158,16 @@ class ClockSampler:
         if not use:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
         reasons = set()
+        bits = 0
         for _, _, r in use:
+            bits |= r
             for bit, name in self.REASONS.items():
                 if r & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(use), "in_timed_region": bool(inside), "source": "nvml"}
+        mhz = sorted(s[1] for s in use)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "sm_mhz_min": mhz[0],
+                "sm_mhz_p90": mhz[int(0.9 * (len(mhz) - 1))], "reasons": sorted(reasons), "reason_bits": hex(bits),
+                "samples": len(use), "in_timed_region": bool(inside), "source": "nvml"}
 
 
 def to_dev(a, device):
@@ -337,6 +342,16 @@ class Mla:
         kept = self.visited - skipped
         return 2 * c["Hq"] * 64 * 576 * self.visited + 2 * c["Hq"] * 64 * 512 * kept
 
+    def host_bytes(self):
+        return self.inp.q.nbytes + self.inp.k.nbytes, self.o.numel() * 2 + self.lse.numel() * 4
+
+    def e2e_call(self, lam, hq, hk, hv, ho, hl):
+        self.q.copy_(hq, non_blocking=True)
+        self.k.copy_(hk, non_blocking=True)
+        self.call(lam)
+        ho.copy_(self.o, non_blocking=True)
+        hl.copy_(self.lse, non_blocking=True)
+
     def rate(self, work, ms):
         return work / (ms * 1e-3) / 1e9
 
@@ -382,7 +397,8 @@ def timed_launches(wl, lam, steps, warmup, flush, sampler=None):
 def e2e_measure(wl, lam, steps, warmup):
     import torch
 
-    hq, hk, hv = to_pinned(wl.inp.q), to_pinned(wl.inp.k), to_pinned(wl.inp.v)
+    hq, hk = to_pinned(wl.inp.q), to_pinned(wl.inp.k)
+    hv = to_pinned(wl.inp.v) if wl.inp.v is not None else None  # MLA: V is the K buffer
     ho = torch.empty(wl.o.shape, dtype=torch.bfloat16).pin_memory()
     hl = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
     wl.count = torch.zeros(1, dtype=torch.int64, device=wl.device)
@@ -483,6 +499,19 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
         kw = dict(scale=inp.scale, causal=True)
         units = lambda r: FLOP_PER_PAIR * (r["n_visited"] * 2 - r["n_skipped"]) / 1e12  # noqa: E731
         unit = "TFLOP/s"
+    elif wl_kind == "mla":
+        c = cfg
+        # per-sequence work is the same at any batch: 4 sequences keep the generator cheap
+        inp = synth.planted_mla(min(4, c["B"]), c["Hq"], c["Lk"], seed=c["seed"], reading="blk")
+        cand = list(range(inp.q.shape[0]))
+        rng.shuffle(cand)
+        kw = dict(scale=inp.scale, causal=False, is_decode=True, num_splits=c["splits"], BN=64, dv=512,
+                  v_row_stride=576)
+        n_tiles = c["B"]
+
+        def units(r):
+            return r["_tiles"] * c["Lk"] * 576 * 2 / 1e9
+        unit = "GB/s"
     else:
         c = cfg
         inp = synth.planted_decode(c["B"], c["Hq"], c["Hkv"], c["Lk"], c["d"], seed=c["seed"], reading="blk")
@@ -499,13 +528,14 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
     # calibrate lambda on the first tiles (their own gaps), then time
     n = max(1, min(len(cand), cores))
     t0 = time.time()
-    r0 = oracle.attention(inp.q, inp.k, inp.v, lam=0.0, tiles=cand[:n], **kw)
+    v = inp.k if inp.v is None else inp.v
+    r0 = oracle.attention(inp.q, inp.k, v, lam=0.0, tiles=cand[:n], **kw)
     dt = time.time() - t0
     lam, _ = oracle.threshold_for_sparsity(r0["gaps"][cand[:n]], r0["visited"][cand[:n]], lam_target)
     n = int(max(1, min(len(cand), n * budget_s / max(dt, 1e-3))))
     tiles = cand[:n]
     t0 = time.time()
-    r = oracle.attention(inp.q, inp.k, inp.v, lam=lam, tiles=tiles, **kw)
+    r = oracle.attention(inp.q, inp.k, v, lam=lam, tiles=tiles, **kw)
     dt = time.time() - t0
     r["_tiles"] = len(tiles)
     return dict(value=units(r) / dt, unit=unit, cores=cores, kind="oracle",
@@ -596,8 +626,8 @@ def aggregate(units_local, seconds_local, world):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    wl_kind = "prefill" if args.workload == "prefill" else "decode"
-    cfg = SIZES[args.size][0] if wl_kind == "prefill" else SIZES[args.size][1]
+    wl_kind = args.workload
+    cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2}[wl_kind]]
     per_step = []
     vals = []
     budget = float(os.environ.get("BLASST_REF_STEP_SECONDS", "8"))
@@ -607,7 +637,7 @@ def run_reference(args, world, rank):
             per_step.append(r["seconds"])
             vals.append(r["value"])
     value = statistics.mean(vals)
-    unit = "TFLOP/s" if wl_kind == "prefill" else "GB/s"
+    unit = r["unit"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(per_step),
@@ -628,7 +658,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--workload", choices=["prefill", "decode"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "decode", "mla"], default="prefill")
     ap.add_argument("--size", choices=sorted(SIZES), default="full",
                     help="full = the benchmark shapes; medium = profiling size; quick = smoke-testing the bench")
     ap.add_argument("--no-sweep", action="store_true")
@@ -662,25 +692,24 @@ def main():
     pcfg, dcfg, mcfg = SIZES[args.size]
     headline_kind = args.workload
     wls = {}
-    try:
-        wls["prefill"] = Prefill(pcfg, dev)
-        wls["prefill"].count = torch.zeros(1, dtype=torch.int64, device=dev)
-        wls["prefill"].call(0.0)
-        torch.cuda.synchronize()
-    except bl.BlasstError as e:
-        if e.status != 2:
-            raise
-        wls.pop("prefill", None)
-        notes.append("prefill kernel not available in this build; headline falls back to decode")
-        headline_kind = "decode"
-    if headline_kind == "decode" or not args.no_sweep:
+    if headline_kind == "prefill":
+        try:
+            wls["prefill"] = Prefill(pcfg, dev)
+            wls["prefill"].count = torch.zeros(1, dtype=torch.int64, device=dev)
+            wls["prefill"].call(0.0)
+            torch.cuda.synchronize()
+        except bl.BlasstError as e:
+            if e.status != 2:
+                raise
+            wls.pop("prefill", None)
+            notes.append("prefill kernel not available in this build; headline falls back to decode")
+            headline_kind = "decode"
+    if headline_kind == "decode":
         wls["decode"] = Decode(dcfg, dev)
-    if not args.no_sweep and not args.no_mla:
+    if headline_kind == "mla":
         wls["mla"] = Mla(mcfg, dev)
-    if not args.no_sweep and args.size == "full" and "prefill" in wls and not args.no_64k:
-        wls["prefill_64k"] = Prefill(PREFILL_64K, dev)
-
-    lams = {k: lambdas_for_targets(w, w.calibrate()) for k, w in wls.items()}
+    # the headline workload is calibrated and timed before any other workload runs
+    lams = {headline_kind: lambdas_for_targets(wls[headline_kind], wls[headline_kind].calibrate())}
 
     # ---- headline: the ~75% point of the headline workload
     wl = wls[headline_kind]
@@ -711,16 +740,31 @@ def main():
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_source": f"{peak_src} copy bandwidth"}
 
-    prof = load_profile_counters("prefill" if wl.bound == "tensor" else "decode")
+    prof = load_profile_counters(wl.kind)
     roof["traffic"] = prof.get("dram_bytes_per_launch")
     if wl.bound == "tensor":
         roof["tensor_pipe_active_pct_ncu"] = prof.get("tensor_pipe_active_pct")
     if prof:
         roof["ncu_source"] = prof.get("source")
 
-    # ---- sweep: 0/50/75% on both workloads, speedup over lambda = 0
+    # ---- sweep: 0/50/75% on every workload, speedup over lambda = 0
     sweep = {}
     if not args.no_sweep:
+        if "prefill" not in wls:
+            try:
+                wls["prefill"] = Prefill(pcfg, dev)
+            except bl.BlasstError as e:
+                if e.status != 2:
+                    raise
+        if "decode" not in wls:
+            wls["decode"] = Decode(dcfg, dev)
+        if "mla" not in wls and not args.no_mla:
+            wls["mla"] = Mla(mcfg, dev)
+        if args.size == "full" and "prefill" in wls and not args.no_64k:
+            wls["prefill_64k"] = Prefill(PREFILL_64K, dev)
+        for k, w in wls.items():
+            if k not in lams:
+                lams[k] = lambdas_for_targets(w, w.calibrate())
         for kind, w in wls.items():
             rows = {}
             base = None

@@ -176,23 +176,12 @@ __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// ------------------------------------------------------------------ tcgen05
-// Shared-memory matrix descriptor for a tile stored with the 128-byte swizzle
-// (SBO = 1024 B between 8-row groups).  K-major operands: LBO unused (1).
-// MN-major operands: LBO = byte distance between 64-element MN blocks.
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo_bytes) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
-    d |= (uint64_t)((1024 >> 4) & 0x3FFF) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-    d |= (uint64_t)2 << 61;  // 128-byte swizzle
-    return d;
-}
-
-// The same descriptor split in halves.  The high half (SBO, version, swizzle)
-// is common to every tile here; the low half holds the start address (16-byte
-// units, bits 0-13) and LBO, so advancing within a tile is a 32-bit add that
+// tcgen05 shared-memory matrix descriptor for a 128-byte-swizzled tile, as two
+// 32-bit halves.  Low half: start address in 16-byte units (bits 0-13) and the
+// leading-dimension byte offset (bits 16-29).  High half: stride-dimension byte
+// offset 1024 (8 rows of 128 B), the sm_100 descriptor version (bit 46 of the
+// whole) and swizzle mode 2 (128 B, bits 61-63).  The high half is common to
+// every tile here; advancing within a tile is a 32-bit add to the low half that
 // never carries out of the address field (shared memory is < 256 KB).
 __host__ __device__ constexpr uint32_t umma_desc_hi_sw128() {
     return (uint32_t)((1024 >> 4) & 0x3FFF) | (1u << 14) | (2u << 29);
@@ -228,15 +217,6 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
 // D[tmem] (+)= A[smem desc] * B[smem desc], descriptors given as halves.
 __device__ __forceinline__ void umma_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t desc_hi,
@@ -262,15 +242,6 @@ __device__ __forceinline__ void umma_ts2(uint32_t d_tmem, uint32_t a_tmem, uint3
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
 // mbarrier arrives once all previously issued tcgen05.mma of this thread completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
@@ -324,65 +295,6 @@ __device__ __forceinline__ bool bar_and(int id, int nthreads, bool pred) {
 
 __device__ __forceinline__ void bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// ----------------------------------------------------------- thread-block clusters
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Address of the same shared-memory location in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// 16 bytes into another CTA's shared memory; completes bytes on that CTA's mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t remote_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     remote_addr),
-                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
-                 : "memory");
-}
-// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into another
-// CTA's, completing the bytes on that CTA's mbarrier (both remote addresses from mapa).
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, uint32_t local_src, uint32_t bytes,
-                                                  uint32_t remote_bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            remote_dst),
-        "r"(local_src), "r"(bytes), "r"(remote_bar)
-        : "memory");
-}
-// Arrive on an mbarrier in another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait on a local mbarrier whose bytes come from another CTA of the cluster.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    long long t0 = clock64();
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (abort && *abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) return false;
-    }
 }
 
 }  // namespace blasst

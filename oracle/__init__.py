@@ -60,7 +60,7 @@ def _load():
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_longlong, ctypes.c_longlong,
                 ctypes.c_double, ctypes.c_double, ctypes.c_int,
-                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 P, ctypes.c_longlong, P,
                 P, P, P, P, P, P,
             ]
@@ -80,7 +80,7 @@ def num_tiles(is_decode, B, Hq, Hkv, Lq, Lk, BM, BN) -> int:
 
 def attention(q, k, v, *, scale, lam, causal, is_decode=False, num_splits=1, BM=None, BN=None,
               dv=None, k_row_stride=None, v_row_stride=None, Lk=None, tiles=None, forced_skip=None,
-              Hkv=None):
+              Hkv=None, seed_splits=False):
     """Run the oracle.
 
     q: uint16 [B, Hq, Lq, d] bf16 bits.  k, v: uint16 arrays holding
@@ -89,6 +89,8 @@ def attention(q, k, v, *, scale, lam, causal, is_decode=False, num_splits=1, BM=
     (natural log), and per (tile, block) arrays skip, visited (uint8) and gaps
     (f64; +inf on a first block, NaN where not visited), plus the counts.
     ``tiles``: optional list of flat tile indices to compute (others: NaN).
+    ``seed_splits`` (decode): splits after the first start their running max
+    at block 0's row maxima and have no forced first block.
     """
     q = np.ascontiguousarray(q, dtype=np.uint16)
     k = np.ascontiguousarray(k, dtype=np.uint16)
@@ -122,7 +124,7 @@ def attention(q, k, v, *, scale, lam, causal, is_decode=False, num_splits=1, BM=
     rc = _load().blasst_oracle_attention(
         _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Lq, Lk, d, dv, k_row_stride, v_row_stride,
         float(scale), float(lam), int(bool(causal)), BM, BN, int(bool(is_decode)), int(num_splits),
-        _ptr(tiles_arr), 0 if tiles_arr is None else len(tiles_arr), _ptr(fs),
+        int(bool(seed_splits)), _ptr(tiles_arr), 0 if tiles_arr is None else len(tiles_arr), _ptr(fs),
         _ptr(o), _ptr(lse), _ptr(skip), _ptr(visited), _ptr(gaps), _ptr(counts))
     if rc != 0:
         raise ValueError(f"oracle returned {rc}")

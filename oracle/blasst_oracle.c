@@ -30,6 +30,11 @@
  * decode splits are independent online-softmax passes over contiguous chunks
  * of ceil(nb/num_splits) blocks, merged exactly on lse; lse = M + ln(l) over
  * kept blocks, natural log.
+ * Split seeding (decode, optional; not on the pages): every split after the
+ * first starts its running max at the row maxima of block 0 instead of -inf
+ * and has no forced first block.  Block 0 then adds nothing to that split's l
+ * or O; only its maxima enter the comparison.  This is the single-pass rule
+ * with the blocks between block 0 and the split start left out of the max.
  *
  * Everything is fp64: bf16 inputs are widened exactly.  Parallel over tiles
  * with OpenMP; each tile's arithmetic is a plain sequential loop nest.
@@ -85,7 +90,7 @@ static int run_tile(long long tile, const uint16_t *q, const uint16_t *k, const 
                     int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv,
                     long long k_row_stride, long long v_row_stride,
                     double scale, double lambda, int causal, int BM, int BN, int is_decode, int num_splits,
-                    int tiles_per_head, int nb, const uint8_t *forced_skip,
+                    int seed_splits, int tiles_per_head, int nb, const uint8_t *forced_skip,
                     double *o, double *lse, uint8_t *skip, uint8_t *visited, double *gaps,
                     long long *n_skipped, long long *n_visited)
 {
@@ -158,6 +163,24 @@ static int run_tile(long long tile, const uint16_t *q, const uint16_t *k, const 
             for (int x = 0; x < dv; x++) acc[(size_t)r * dv + x] = 0.0;
         }
         int first = 1;
+        if (is_decode && seed_splits && sp > 0 && j0 < j1) {
+            /* seed: the running max starts at block 0's row maxima */
+            for (int r = 0; r < nrows; r++) {
+                int last_key = causal ? row_pos[r] + (Lk - Lq) : Lk - 1;
+                double m = -INFINITY;
+                for (int cc = 0; cc < BN; cc++) {
+                    int key = cc;
+                    if (key < Lk && key <= last_key) {
+                        const uint16_t *kp = kbase + (long long)key * k_row_stride;
+                        double dot = 0.0;
+                        for (int x = 0; x < d; x++) dot += qrow[(size_t)r * d + x] * bf16_to_double(kp[x]);
+                        if (scale * dot > m) m = scale * dot;
+                    }
+                }
+                M[r] = m;
+            }
+            first = 0;
+        }
         for (int j = j0; j < j1; j++) {
             long long pair = tile * nb + j;
             /* scores of the block; masked entries are -inf */
@@ -273,6 +296,8 @@ static int run_tile(long long tile, const uint16_t *q, const uint16_t *k, const 
  *     tiles are left untouched.
  * forced_skip [n_tiles_total * nb] or NULL: use this skip decision instead of
  *     the rule (marking a first block is an error, ORACLE_BAD_FORCED).
+ * seed_splits: decode only; nonzero seeds the running max of every split
+ *     after the first with block 0's row maxima (see the header).
  * Outputs: o [B, Hq, Lq, dv], lse [B, Hq, Lq] (natural log), and per
  *     (tile, block) pair: skip (1 = skipped), visited (1 = at least one
  *     unmasked score), gaps (max over voting rows of m~ - m; +inf on a first
@@ -284,7 +309,7 @@ int blasst_oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t
                             int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv,
                             long long k_row_stride, long long v_row_stride,
                             double scale, double lambda, int causal,
-                            int BM, int BN, int is_decode, int num_splits,
+                            int BM, int BN, int is_decode, int num_splits, int seed_splits,
                             const long long *tiles, long long n_tiles, const uint8_t *forced_skip,
                             double *o, double *lse, uint8_t *skip, uint8_t *visited, double *gaps,
                             long long *counts)
@@ -311,7 +336,8 @@ int blasst_oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t
         long long tile = tiles ? tiles[i] : i;
         long long sk = 0, vi = 0;
         int st = run_tile(tile, q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, k_row_stride, v_row_stride, scale, lambda,
-                          causal, BM, BN, is_decode, num_splits, tph, nb, forced_skip, o, lse, skip, visited,
+                          causal, BM, BN, is_decode, num_splits, seed_splits, tph, nb, forced_skip, o, lse, skip,
+                          visited,
                           gaps, &sk, &vi);
         skipped += sk;
         vis += vi;

@@ -67,11 +67,14 @@ def tile_rows(is_decode, Hq, Hkv, Lq, BM, tile):
     return b, rows
 
 
-def closed_form_decisions(q, k, scale, causal, lam, BM, BN, is_decode=False, num_splits=1, d=None):
+def closed_form_decisions(q, k, scale, causal, lam, BM, BN, is_decode=False, num_splits=1, d=None,
+                          seed_splits=False):
     """Skip mask from per-block row maxima only (prefix-max form).
 
     skip_j <=> j is not the first visited block of its split and
     max over voting rows r of (m~_rj - max_{j' <= j in split} m~_rj') < ln(lam).
+    With seed_splits (decode), block 0's row maxima join the prefix max of every
+    later split, which then has no forced first block.
     Returns (skip, visited) as [n_tiles, nb] uint8.
     """
     B, Hq, Lq, _ = q.shape
@@ -106,11 +109,15 @@ def closed_form_decisions(q, k, scale, causal, lam, BM, BN, is_decode=False, num
             j0, j1 = sp * per, min(nb, (sp + 1) * per)
             if j0 >= j1:
                 continue
-            pm = np.maximum.accumulate(mt[:, j0:j1], axis=1)
+            seeded = is_decode and seed_splits and sp > 0
+            if seeded:
+                pm = np.maximum.accumulate(np.concatenate([mt[:, :1], mt[:, j0:j1]], axis=1), axis=1)[:, 1:]
+            else:
+                pm = np.maximum.accumulate(mt[:, j0:j1], axis=1)
             with np.errstate(invalid="ignore"):
                 gap = np.where(np.isfinite(mt[:, j0:j1]), mt[:, j0:j1] - pm, -np.inf).max(axis=0)
             v = vis[j0:j1]
-            first = np.argmax(v) if v.any() else None
+            first = np.argmax(v) if v.any() and not seeded else None
             dec = v & (gap < ln_lam)
             if first is not None:
                 dec[first] = False

@@ -111,7 +111,7 @@ def test_hand_cases(case, cl):
     lam = math.exp(cl["ln_lambda"]) if "ln_lambda" in cl else cl["lambda"]
     r = oracle.attention(q, k, v, scale=1.0, lam=lam, causal=case["causal"],
                          is_decode=case["mode"] == "decode", num_splits=case.get("num_splits", 1),
-                         BM=case["BM"], BN=case["BN"])
+                         BM=case["BM"], BN=case["BN"], seed_splits=case.get("seed_splits", False))
     assert r["skip"].tolist() == cl["skip"]
     assert r["visited"].tolist() == cl["visited"]
     if "lse" in cl:
@@ -241,6 +241,58 @@ def test_splits_restart_running_max():
     firsts = r["skip"][0, ::8]
     assert np.all(firsts == 0)
     assert r["n_skipped"] > 0
+
+
+# ---------------------------------------------------------------------------
+# split seeding (decode): later splits start their running max at block 0's maxima
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("splits", [2, 5, 16])
+def test_seeded_dense_decode_matches_bruteforce(splits):
+    # at lambda = 0 nothing is skipped: the seed only moves the exp reference
+    inp = planted_decode(2, 8, 2, 1500, 32, Lq=2, seed=21, reading="blk")
+    r = _run(inp, 0.0, True, is_decode=True, num_splits=splits, seed_splits=True)
+    O, LSE = dense_attention(inp.q, inp.k, inp.v, inp.scale, True)
+    np.testing.assert_allclose(r["o"], O, atol=1e-9, rtol=0)
+    np.testing.assert_allclose(r["lse"], LSE, atol=1e-9, rtol=0)
+
+
+@pytest.mark.parametrize("lam", [1e-3, 0.02, 0.2, 0.9])
+@pytest.mark.parametrize("splits", [2, 4, 16])
+def test_seeded_mask_equals_prefix_max_closed_form(lam, splits):
+    inp = planted_decode(2, 8, 2, 1024, 32, Lq=2, seed=9, reading="blk")
+    r = _run(inp, lam, True, is_decode=True, num_splits=splits, BN=64, seed_splits=True)
+    skip, vis = closed_form_decisions(inp.q, inp.k, inp.scale, True, lam, 128, 64, is_decode=True,
+                                      num_splits=splits, seed_splits=True)
+    assert np.array_equal(r["visited"], vis)
+    assert np.array_equal(r["skip"], skip)
+
+
+def test_seeded_outputs_equal_masked_softmax():
+    # block 0 enters later splits only through its maxima, never through l or O
+    inp = planted_decode(1, 4, 1, 2048, 32, seed=4, reading="blk")
+    r = _run(inp, 0.05, False, is_decode=True, num_splits=8, BN=64, seed_splits=True)
+    assert r["n_skipped"] > 0
+    O, LSE = masked_attention(inp.q, inp.k, inp.v, inp.scale, False, r["skip"], 128, 64, is_decode=True)
+    np.testing.assert_allclose(r["o"], O, atol=1e-9, rtol=0)
+    np.testing.assert_allclose(r["lse"], LSE, atol=1e-9, rtol=0)
+
+
+def test_seeded_one_split_is_unseeded():
+    inp = planted_decode(2, 8, 2, 1024, 32, seed=3, reading="blk")
+    a = _run(inp, 0.1, False, is_decode=True, num_splits=1, seed_splits=True)
+    b = _run(inp, 0.1, False, is_decode=True, num_splits=1)
+    assert np.array_equal(a["skip"], b["skip"])
+    np.testing.assert_array_equal(a["o"], b["o"])
+
+
+@pytest.mark.parametrize("lam", [0.005, 0.05, 0.5])
+def test_seeded_skips_contain_unseeded(lam):
+    # the seed can only raise the running max, so every gap shrinks or stays
+    inp = planted_decode(2, 8, 2, 4096, 32, seed=11, reading="blk")
+    a = _run(inp, lam, False, is_decode=True, num_splits=16, seed_splits=True)
+    b = _run(inp, lam, False, is_decode=True, num_splits=16)
+    assert np.all(b["skip"] <= a["skip"])
+    assert a["n_skipped"] > b["n_skipped"]
 
 
 # ---------------------------------------------------------------------------

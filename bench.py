@@ -240,6 +240,7 @@ class Decode:
     kind = "decode"
     unit = "GB/s"
     bound = "hbm"
+    seed_splits = False
 
     def __init__(self, cfg, device):
         import synth
@@ -263,13 +264,13 @@ class Decode:
 
     def calibrate(self):
         gaps, _, _ = self.bl.calibrate(self.q, self.k, scale=self.inp.scale, causal=False, mode="decode",
-                                       num_splits=self.cfg["splits"])
+                                       num_splits=self.cfg["splits"], seed_splits=self.seed_splits)
         return gaps.cpu().numpy()
 
     def call(self, lam, stream=None):
         return self.bl.decode(self.q, self.k, self.v, scale=self.inp.scale, lam=lam, num_splits=self.cfg["splits"],
                               o=self.o, lse=self.lse, skip_mask=False, skip_count=self.count, workspace=self.ws,
-                              stream=stream)
+                              stream=stream, seed_splits=self.seed_splits)
 
     def work(self, skipped):
         c = self.cfg
@@ -293,6 +294,15 @@ class Decode:
         self.call(lam)
         ho.copy_(self.o, non_blocking=True)
         hl.copy_(self.lse, non_blocking=True)
+
+
+class DecodeSeeded(Decode):
+    """The same decode with split seeding: splits after the first start their
+    running max at block 0's row maxima.  Effective bytes are counted as for
+    Decode (the extra block-0 read of each split is overhead, not work)."""
+
+    kind = "decode_seeded"
+    seed_splits = True
 
 
 class Mla:
@@ -366,6 +376,7 @@ def lambdas_for_targets(wl, gaps):
         if ach + 0.02 < t:  # unreachable target: the highest reachable sparsity
             lam, ach = wl.bl.calibrate_threshold(gaps, 1.0)
         out[t] = (lam, ach)
+    out["max"] = wl.bl.calibrate_threshold(gaps, 1.0)  # (lambda, sparsity) as lambda -> 1
     return out
 
 
@@ -666,6 +677,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mla", action="store_true")
     ap.add_argument("--no-64k", action="store_true")
+    ap.add_argument("--no-seeded", action="store_true", help="skip the split-seeded decode rows of the sweep")
     ap.add_argument("--calibration", action="store_true",
                     help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
     args = ap.parse_args()
@@ -758,6 +770,10 @@ def main():
                     raise
         if "decode" not in wls:
             wls["decode"] = Decode(dcfg, dev)
+        if not args.no_seeded:
+            ws = DecodeSeeded.__new__(DecodeSeeded)  # shares the decode workload's inputs and buffers
+            ws.__dict__.update(wls["decode"].__dict__)
+            wls["decode_seeded"] = ws
         if "mla" not in wls and not args.no_mla:
             wls["mla"] = Mla(mcfg, dev)
         if args.size == "full" and "prefill" in wls and not args.no_64k:
@@ -786,6 +802,7 @@ def main():
                 if hasattr(w, "flops"):
                     tf = w.flops(sk) / (med * 1e-3) / 1e12
                     rows[f"{int(t * 100)}%"].update(tflops=tf, tensor_frac_of_measured_peak=tf / peaks["bf16_tflops"])
+            rows["max_reachable_sparsity"] = lams[kind]["max"][1]
             sweep[kind] = rows
 
     # ---- calibration fit across context lengths (prefill-shaped decision pass)

@@ -46,6 +46,7 @@ class Opts(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("gaps_out", ctypes.c_void_p),
         ("status_word", ctypes.c_void_p),
+        ("seed_splits", ctypes.c_int),
     ]
 
     def __init__(self, **kw):
@@ -168,7 +169,7 @@ def prefill(q, k, v, *, scale, lam=0.0, causal=True, o=None, lse=None, skip_mask
 
 
 def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o=None, lse=None,
-           skip_mask=True, skip_count=True, workspace=None, status_word=None, stream=None):
+           skip_mask=True, skip_count=True, workspace=None, status_word=None, stream=None, seed_splits=False):
     """Split-KV decode with block skipping.
 
     GQA/MQA: q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA (16 splits by default).
@@ -176,6 +177,8 @@ def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o
     the first 512 columns of each cache row; 2 splits by default).
     Returns (o, lse, skip_mask [B*Hkv, W] int32 or None, skip_count [1] int64 or None).
     ``workspace``: optional uint8 CUDA tensor of at least decode_workspace_bytes() bytes.
+    ``seed_splits`` (d = 128): splits after the first start their running max at
+    block 0's row maxima and have no forced first block.
     """
     import torch
 
@@ -189,7 +192,8 @@ def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
     opts = Opts(num_splits=num_splits or 0, dv=dv, k_row_stride=krs, v_row_stride=vrs,
-                status_word=None if status_word is None else status_word.data_ptr())
+                status_word=None if status_word is None else status_word.data_ptr(),
+                seed_splits=int(bool(seed_splits)))
     if workspace is not None:
         opts.workspace = workspace.data_ptr()
         opts.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -228,7 +232,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=None, dv=None, skip_mask=True,
-              skip_count=True, stream=None):
+              skip_count=True, stream=None, seed_splits=False):
     """Decision-only pass.  Returns (gaps [tiles, nb] fp32, skip_mask, skip_count)."""
     import torch
 
@@ -246,7 +250,8 @@ def calibrate(q, k, *, scale, lam=0.0, causal=True, mode="prefill", num_splits=N
     else:
         raise ValueError(mode)
     gaps = torch.empty((tiles, nb), dtype=torch.float32, device=q.device)
-    opts = Opts(mode=m, num_splits=num_splits or 0, gaps_out=gaps.data_ptr(), dv=dv or 0)
+    opts = Opts(mode=m, num_splits=num_splits or 0, gaps_out=gaps.data_ptr(), dv=dv or 0,
+                seed_splits=int(bool(seed_splits)))
     mk, c = _attn("blasst_calibrate", q, k, None, scale=scale, lam=lam, causal=causal, o=None, lse=None,
                   want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=tiles,
                   n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=d)

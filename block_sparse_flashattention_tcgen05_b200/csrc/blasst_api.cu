@@ -203,6 +203,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         return BLASST_ERR_INVALID;
     }
     if (op.block_n != 0 && op.block_n != kDecodeBlockN) return BLASST_ERR_UNSUPPORTED;
+    if (op.seed_splits && d != 128) return BLASST_ERR_UNSUPPORTED;  // split seeding: GQA/MQA decode only
     if (d == 576) return run_mla(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count,
                                  stream, op, c, calib);
     if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
@@ -267,6 +268,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     p.causal = causal ? 1 : 0;
     p.scale_log2 = (float)(scale * kLog2e);
     p.thr_log2 = log2_threshold(lambda);
+    p.seed = op.seed_splits ? 1 : 0;
     e = launch_decode(p, tk, tv, calib, R <= 8 ? 1 : 2, sm);
     if (e != cudaSuccess) return cuda_fail(e, "decode split kernel");
     if (!calib) {
@@ -296,6 +298,7 @@ blasst_status run_prefill(const void *q, const void *k, const void *v, void *o, 
     Common c;
     blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, op, &c);
     if (st != BLASST_OK) return st;
+    if (op.seed_splits) return BLASST_ERR_UNSUPPORTED;  // prefill has no splits
     if (!calib) {
         if (!v || !o || !lse) return BLASST_ERR_INVALID;
         if (!aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4)) return BLASST_ERR_INVALID;

@@ -20,8 +20,10 @@
 //              conditional V loads after the key blocks).
 //
 // The running max per row restarts in every split; the first visited block
-// of a split is always kept.  Scores are handled in log2 units:
-// s2 = (q.k) * scale * log2(e), compared with log2(lambda).
+// of a split is always kept.  With split seeding, every split after the first
+// instead starts from the row maxima of block 0 (one extra K block through the
+// ring, no decision, no V) and has no forced first block.  Scores are handled
+// in log2 units: s2 = (q.k) * scale * log2(e), compared with log2(lambda).
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -78,6 +80,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int j1 = min(p.nb, j0 + p.per_split);
     const int nblk = max(0, j1 - j0);
     const int bh = b * p.Hkv + hkv;
+    // ring entries: [block 0 (seed)], then the split's blocks j0 .. j1-1
+    const int seed = (p.seed && split > 0 && nblk > 0) ? 1 : 0;
+    const int nent = nblk + seed;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NK; i++) {
@@ -101,16 +106,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane != 0) return;
         tma_prefetch_desc(&tmap_k);
         int issued = 0;
-        for (int jj = 0; jj < nblk; jj++) {
-            const int slot = jj % NK;
-            if (jj >= NK && !mbar_wait(&tl->k_empty[slot], ((jj / NK) & 1) ^ 1, &tl->abort)) {
+        for (int e = 0; e < nent; e++) {
+            const int slot = e % NK;
+            if (e >= NK && !mbar_wait(&tl->k_empty[slot], ((e / NK) & 1) ^ 1, &tl->abort)) {
                 set_timeout(tl, p.status);
                 break;
             }
+            const int blk = (seed && e == 0) ? 0 : j0 + e - seed;
             uint8_t *dst = kring + slot * kStageBytes;
             mbar_arrive_expect_tx(&tl->k_full[slot], kStageBytes);
-            tma_load_3d(dst, &tmap_k, &tl->k_full[slot], 0, (j0 + jj) * kDecodeBlockN, bh);
-            tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, (j0 + jj) * kDecodeBlockN, bh);
+            tma_load_3d(dst, &tmap_k, &tl->k_full[slot], 0, blk * kDecodeBlockN, bh);
+            tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, blk * kDecodeBlockN, bh);
             issued++;
         }
         if (tl->abort) {  // let copies in flight land before the CTA exits
@@ -204,10 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned long long n_skip = 0;
     const float NEG_INF = -CUDART_INF_F;
 
-    for (int jj = 0; jj < nblk; jj++) {
-        const int j = j0 + jj;
-        const int slot = jj % NK;
-        if (!mbar_wait(&tl->k_full[slot], (jj / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
+    for (int e = 0; e < nent; e++) {
+        const int jj = e - seed;  // block index within the split; -1: the seed block
+        const int j = jj < 0 ? 0 : j0 + jj;
+        const int slot = e % NK;
+        if (!mbar_wait(&tl->k_full[slot], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
         const uint8_t *kb = kring + slot * kStageBytes;
 
         float acc[NT][4];
@@ -248,11 +255,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (g4 == 0) {
 #pragma unroll
             for (int nt = 0; nt < NT; nt++) {
-                tl->red[jj & 1][warp][nt * 8 + 2 * t4] = cmax[nt][0];
-                tl->red[jj & 1][warp][nt * 8 + 2 * t4 + 1] = cmax[nt][1];
+                tl->red[e & 1][warp][nt * 8 + 2 * t4] = cmax[nt][0];
+                tl->red[e & 1][warp][nt * 8 + 2 * t4 + 1] = cmax[nt][1];
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+
+        if (jj < 0) {
+            // the seed block: its row maxima start the running max of this split
+#pragma unroll
+            for (int c = 0; c < NC; c++) {
+                float mt = tl->red[e & 1][0][c];
+#pragma unroll
+                for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 1][w][c]);
+                Mall[c] = mt;
+            }
+            seen = true;  // no forced first block after a seed
+            continue;
+        }
 
         // block row maxima of the whole tile, running max after the block, gap
         float Mn[NC];
@@ -260,9 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool visited = false;
 #pragma unroll
         for (int c = 0; c < NC; c++) {
-            float mt = tl->red[jj & 1][0][c];
+            float mt = tl->red[e & 1][0][c];
 #pragma unroll
-            for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[jj & 1][w][c]);
+            for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 1][w][c]);
             Mn[c] = fmaxf(Mall[c], mt);
             if (mt > NEG_INF) {
                 visited = true;

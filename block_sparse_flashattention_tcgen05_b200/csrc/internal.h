@@ -26,6 +26,7 @@ struct DecodeParams {
     int causal;
     float scale_log2;               // scale * log2(e)
     float thr_log2;                 // log2(lambda), -inf for lambda = 0
+    int seed;                       // 1: splits after the first start from block 0's row maxima
 };
 
 struct CombineParams {

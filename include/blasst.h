@@ -93,6 +93,16 @@ typedef struct blasst_opts {
                                   tile's (split's) first block, NaN if not visited */
     unsigned int *status_word; /* device word the caller zeroes; the library ORs in
                                   a nonzero code when a bounded wait expires */
+    int seed_splits;           /* decode (d = 128) only: nonzero seeds the running
+                                  max of every split after the first with the row
+                                  maxima of block 0, and such a split has no forced
+                                  first block.  Block 0 enters those splits only
+                                  through the comparison (one extra 64-key Q.K^T per
+                                  split); it lifts the cap that restarting the max
+                                  puts on sparsity.  Not a rule of the paper: a
+                                  restatement of its single-pass rule (block 0's
+                                  maxima are part of the running max) for split-KV.
+                                  Other paths return BLASST_ERR_UNSUPPORTED. */
 } blasst_opts;
 
 /*

@@ -83,6 +83,11 @@ def test_decode_unsupported_tile_and_small_workspace(bl):
     assert _call(bl, "blasst_decode", opts=bl.Opts(workspace=FAKE + 16, workspace_bytes=1 << 30)) == 1
 
 
+def test_split_seeding_only_on_gqa_decode(bl):
+    assert _call(bl, "blasst_prefill", opts=bl.Opts(seed_splits=1)) == 2     # prefill has no splits
+    assert _call(bl, "blasst_decode", d=576, opts=bl.Opts(seed_splits=1, dv=512)) == 2  # MLA
+
+
 def test_calibrate_requires_gaps_and_valid_mode(bl):
     assert _call(bl, "blasst_calibrate") == 1                 # no gaps_out
     assert _call(bl, "blasst_calibrate", opts=bl.Opts(mode=7, gaps_out=FAKE)) == 1

@@ -28,9 +28,10 @@ def to_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True, one_hot=False):
+def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True, one_hot=False, seed_splits=False):
     q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
-    o, lse, mask, cnt = bl.decode(q, k, v, scale=inp.scale, lam=lam, causal=causal, num_splits=splits)
+    o, lse, mask, cnt = bl.decode(q, k, v, scale=inp.scale, lam=lam, causal=causal, num_splits=splits,
+                                  seed_splits=seed_splits)
     torch.cuda.synchronize()
     B, Hq, Lq, d = inp.q.shape
     Hkv, Lk = inp.k.shape[1], inp.k.shape[2]
@@ -38,14 +39,14 @@ def check_decode(bl, inp, lam, causal, splits, tiles=None, band_ok=True, one_hot
     bits = unpack_mask(mask.cpu().numpy(), nb)
     assert int(cnt.item()) == int(bits.sum())
     ref = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=lam, causal=causal, is_decode=True,
-                           num_splits=splits, BN=64, tiles=tiles)
+                           num_splits=splits, BN=64, tiles=tiles, seed_splits=seed_splits)
     nd, nband = compare_masks(bits, ref, lam, tiles)
     assert nd == 0, f"{nd} mask bits differ outside the band"
     if not band_ok:
         assert nband == 0
     forced = bits.copy()
     fr = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=lam, causal=causal, is_decode=True,
-                          num_splits=splits, BN=64, tiles=tiles, forced_skip=forced)
+                          num_splits=splits, BN=64, tiles=tiles, forced_skip=forced, seed_splits=seed_splits)
     og = bf16_tensor_to_f64(o)
     lg = lse.cpu().numpy().astype(np.float64)
     rows = None
@@ -173,6 +174,74 @@ def test_decode_calibrate_matches_decode_masks(bl):
     fin = np.isfinite(ref["gaps"])
     assert np.array_equal(np.isinf(g), np.isinf(ref["gaps"]))
     assert np.max(np.abs(g[fin] - ref["gaps"][fin])) < 1e-3
+
+
+# ------------------------------------------------------------- split seeding
+@pytest.mark.parametrize("lam", [0.0, 1e-3, 0.05, 0.5, 0.999])
+@pytest.mark.parametrize("splits", [4, 16])
+def test_decode_seeded(bl, lam, splits):
+    inp = planted_decode(2, 8, 2, 64 * 37 + 13, 128, seed=21, reading="blk")
+    bits, _ = check_decode(bl, inp, lam, False, splits, seed_splits=True)
+    if lam == 0.0:
+        assert bits.sum() == 0
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.1])
+def test_decode_seeded_two_ntiles_causal(bl, lam):
+    inp = planted_decode(1, 8, 1, 3000, 128, Lq=2, seed=3, reading="blk")
+    check_decode(bl, inp, lam, True, 5, seed_splits=True)
+
+
+def test_decode_seeded_short_cache_empty_splits(bl):
+    inp = planted_decode(2, 4, 1, 50, 128, seed=8, reading="lit")
+    check_decode(bl, inp, 0.3, False, 16, seed_splits=True)
+
+
+@pytest.mark.parametrize("name", ["one_row_two_splits_seeded", "one_row_seeded_split_all_skipped"])
+def test_decode_seeded_hand_cases_exact(bl, name):
+    case, q, k, v = _expanded_hand_case(name, 64)
+    from synth import AttnInputs
+
+    inp = AttnInputs(q, k, v, 1.0)
+    for cl in case["cases_lambda"]:
+        lam = math.exp(cl["ln_lambda"]) if "ln_lambda" in cl else cl["lambda"]
+        bits, _ = check_decode(bl, inp, lam, False, case["num_splits"], one_hot=True, seed_splits=True)
+        assert bits.tolist() == cl["skip"]
+
+
+def test_decode_seeded_calibrate_gaps(bl):
+    inp = planted_decode(2, 8, 2, 5000, 128, seed=4, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    gaps, mc, cc = bl.calibrate(q, k, scale=inp.scale, lam=0.05, mode="decode", num_splits=8, seed_splits=True)
+    _, _, md, cd = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=8, seed_splits=True)
+    torch.cuda.synchronize()
+    assert torch.equal(mc, md) and torch.equal(cc, cd)
+    ref = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.05, causal=False, is_decode=True,
+                           num_splits=8, BN=64, seed_splits=True)
+    g = gaps.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(ref["gaps"])
+    assert np.array_equal(np.isinf(g), np.isinf(ref["gaps"]))
+    assert np.max(np.abs(g[fin] - ref["gaps"][fin])) < 1e-3
+
+
+def test_decode_seeded_skips_contain_unseeded(bl):
+    inp = planted_decode(4, 32, 8, 8192, 128, seed=13, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    _, _, m0, c0 = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=16)
+    _, _, m1, c1 = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=16, seed_splits=True)
+    torch.cuda.synchronize()
+    a, b = m0.cpu().numpy().astype(np.uint32), m1.cpu().numpy().astype(np.uint32)
+    assert np.all((a & ~b) == 0)
+    assert int(c1.item()) > int(c0.item())
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("lam", [0.0, 0.05])
+def test_decode_seeded_full_size_sampled(bl, lam):
+    inp = planted_decode(32, 32, 8, 32768, 128, seed=3, reading="blk")
+    rng = np.random.default_rng(1)
+    tiles = np.sort(rng.choice(32 * 8, 8, replace=False))
+    check_decode(bl, inp, lam, False, 16, tiles=tiles, seed_splits=True)
 
 
 @pytest.mark.slow

@@ -781,16 +781,24 @@ def main():
         for k, w in wls.items():
             if k not in lams:
                 lams[k] = lambdas_for_targets(w, w.calibrate())
+        rounds = 4
         for kind, w in wls.items():
             rows = {}
-            base = None
+            # the sparsity points of a workload are timed round-robin, so that a drift of
+            # clocks or temperature during the sweep lands on all of them alike
+            times = {t: [] for t in TARGETS}
+            sk_by_t = {}
+            for rnd in range(rounds):
+                for t in TARGETS:
+                    ms_t, sk_by_t[t] = timed_launches(w, lams[kind][t][0], max(2, args.steps // (2 * rounds)),
+                                                      3 if rnd == 0 else 1, flush)
+                    times[t] += ms_t
+            base = statistics.median(times[0.0])
             for t in TARGETS:
-                lam, ach = lams[kind][t]
-                ms_t, sk = timed_launches(w, lam, max(5, args.steps // 2), 3, flush)
-                med = statistics.median(ms_t)
+                lam = lams[kind][t][0]
+                sk = sk_by_t[t]
+                med = statistics.median(times[t])
                 r = w.rate(w.work(sk), med)
-                if t == 0.0:
-                    base = med
                 pk = peaks["bf16_tflops"] if w.bound == "tensor" else peaks["hbm_gbs"]
                 rows[f"{int(t * 100)}%"] = {
                     "lambda": lam, "a=lambda*L": lam * (w.cfg.get("L") or w.cfg.get("Lk")),

@@ -173,7 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued = 0;
             for (int j = 0; j <= jmax_all && !tl->abort; j++) {
                 const int st = j % kStagesV;
-                if (j >= kStagesV && !mbar_wait(&tl->v_empty[st], ((j / kStagesV) & 1) ^ 1, &tl->abort)) {
+                // the stage is free once the MMA warp is done with its previous block and that
+                // block's load has landed (a block every tile skipped is released unread)
+                if (j >= kStagesV && (!mbar_wait(&tl->v_empty[st], ((j / kStagesV) & 1) ^ 1, &tl->abort) ||
+                                      !mbar_wait(&tl->v_full[st], ((j / kStagesV) & 1) ^ 1, &tl->abort))) {
                     set_timeout(tl, p.status);
                     break;
                 }
@@ -182,10 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(sv + st * kTileBytes + kBoxBytes, &tmap_v, &tl->v_full[st], 64, j * 128, kvrow);
                 issued++;
             }
-            if (tl->abort) {
-                for (int j = max(0, issued - kStagesV); j < issued; j++)
-                    mbar_wait(&tl->v_full[j % kStagesV], (j / kStagesV) & 1, nullptr);
-            }
+            // loads nobody waited for (blocks every tile skipped, or an abort) land before exit
+            for (int j = max(0, issued - kStagesV); j < issued; j++)
+                mbar_wait(&tl->v_full[j % kStagesV], (j / kStagesV) & 1, nullptr);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -269,12 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 if (!CALIB) {
-                    // consume V_j's load even when every tile skipped the block, so the
-                    // slot's barrier phase is complete before the producer refills it
-                    if (!v_waited && !mbar_wait(&tl->v_full[st], (j / kStagesV) & 1, &tl->abort)) {
-                        set_timeout(tl, p.status);
-                        break;
-                    }
+                    // V_j's stage goes back to the producer after the P.V that read it; when
+                    // every tile skipped block j nothing here waits for its load (the producer
+                    // does, before refilling the stage)
                     umma_commit(&tl->v_empty[st]);
                 }
                 if (k_next_waited) umma_commit(&tl->k_empty[(j + 1) % kStagesK]);

@@ -305,6 +305,96 @@ class DecodeSeeded(Decode):
     seed_splits = True
 
 
+class DecodePaged:
+    """Decode over a paged, ragged cache: the batch-32 GQA decode's keys, each
+    sequence cut to its own length (uniform in [min_len, Lk], seeded) and
+    scattered into randomly ordered 64-key pages.  Effective bytes: each
+    sequence's own keys, kept V blocks, q and o."""
+
+    kind = "decode_paged"
+    unit = "GB/s"
+    bound = "hbm"
+
+    def __init__(self, src, device, min_len=8192, seed=11):
+        import numpy as np
+        import torch
+
+        self.bl = src.bl
+        self.device = device
+        c = src.cfg
+        self.cfg = dict(c, workload=f"decode GQA, paged 64-key cache, lengths {min_len}..{c['Lk']}, 16 splits",
+                        min_len=min_len)
+        self.inp = src.inp
+        B, Hkv, L, d = src.inp.k.shape
+        assert L % 64 == 0, "the cache length must be whole pages"
+        rng = np.random.default_rng(seed)
+        self.lens = rng.integers(min_len, L + 1, size=B).astype(np.int32)
+        npg = (self.lens + 63) // 64
+        num_pages = int(npg.sum())
+        order = rng.permutation(num_pages).astype(np.int32)
+        max_pages = (L + 63) // 64
+        table = np.zeros((B, max_pages), np.int32)
+        kp = torch.empty((num_pages, Hkv, 64, d), dtype=torch.bfloat16, device=device)
+        vp = torch.empty_like(kp)
+        at = 0
+        for b in range(B):
+            n = int(npg[b])
+            ids = order[at:at + n]
+            at += n
+            table[b, :n] = ids
+            idx = torch.from_numpy(ids.astype(np.int64)).to(device)
+            kp[idx] = src.k[b, :, : n * 64].reshape(Hkv, n, 64, d).transpose(0, 1)
+            vp[idx] = src.v[b, :, : n * 64].reshape(Hkv, n, 64, d).transpose(0, 1)
+        self.kp, self.vp = kp, vp
+        self.table = torch.from_numpy(table).to(device)
+        self.lens_dev = torch.from_numpy(self.lens).to(device)
+        self.q, self.o, self.lse, self.ws = src.q, src.o, src.lse, src.ws
+        self.visited = int(Hkv * npg.sum())
+        self.key_bytes = int(Hkv * self.lens.sum()) * d * 2
+        self.launches = 2
+
+    def call(self, lam, stream=None):
+        return self.bl.decode_paged(self.q, self.kp, self.vp, self.table, self.lens_dev, scale=self.inp.scale, lam=lam,
+                                    num_splits=self.cfg["splits"], o=self.o, lse=self.lse, skip_mask=False,
+                                    skip_count=self.count, workspace=self.ws, stream=stream)
+
+    def lambdas(self):
+        """lambda for each target by bisection on the measured skip count (monotone in lambda)."""
+        import math
+
+        import torch
+
+        self.count = torch.zeros(1, dtype=torch.int64, device=self.device)
+
+        def frac(lam):
+            self.call(lam)
+            torch.cuda.synchronize()
+            return int(self.count.item()) / self.visited
+
+        top = frac(1 - 1e-7)
+        out = {0.0: (0.0, 0.0), "max": (1 - 1e-7, top)}
+        for t in TARGETS[1:]:
+            if top + 0.02 < t:
+                out[t] = (1 - 1e-7, top)
+                continue
+            lo, hi = math.log(1e-9), math.log(1 - 1e-7)
+            for _ in range(22):
+                mid = 0.5 * (lo + hi)
+                if frac(math.exp(mid)) < t:
+                    lo = mid
+                else:
+                    hi = mid
+            out[t] = (math.exp(hi), frac(math.exp(hi)))
+        return out
+
+    def work(self, skipped):
+        kept = self.visited - skipped
+        return self.key_bytes + kept * 64 * 128 * 2 + self.inp.q.nbytes * 2 + self.lse.numel() * 4
+
+    def rate(self, work, ms):
+        return work / (ms * 1e-3) / 1e9
+
+
 class Mla:
     """MLA decode: 576-column latent cache (V = first 512 columns), all heads in one tile."""
 
@@ -678,6 +768,7 @@ def main():
     ap.add_argument("--no-mla", action="store_true")
     ap.add_argument("--no-64k", action="store_true")
     ap.add_argument("--no-seeded", action="store_true", help="skip the split-seeded decode rows of the sweep")
+    ap.add_argument("--no-paged", action="store_true", help="skip the paged, ragged decode rows of the sweep")
     ap.add_argument("--calibration", action="store_true",
                     help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
     args = ap.parse_args()
@@ -774,13 +865,16 @@ def main():
             ws = DecodeSeeded.__new__(DecodeSeeded)  # shares the decode workload's inputs and buffers
             ws.__dict__.update(wls["decode"].__dict__)
             wls["decode_seeded"] = ws
+        if not args.no_paged:
+            wls["decode_paged"] = DecodePaged(wls["decode"], dev,
+                                              min_len=min(8192, wls["decode"].cfg["Lk"] // 4))
         if "mla" not in wls and not args.no_mla:
             wls["mla"] = Mla(mcfg, dev)
         if args.size == "full" and "prefill" in wls and not args.no_64k:
             wls["prefill_64k"] = Prefill(PREFILL_64K, dev)
         for k, w in wls.items():
             if k not in lams:
-                lams[k] = lambdas_for_targets(w, w.calibrate())
+                lams[k] = w.lambdas() if hasattr(w, "lambdas") else lambdas_for_targets(w, w.calibrate())
         rounds = 4
         for kind, w in wls.items():
             rows = {}

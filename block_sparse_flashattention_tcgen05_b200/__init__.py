@@ -76,6 +76,10 @@ def lib() -> ctypes.CDLL:
             f = getattr(L, name)
             f.restype = ctypes.c_int
             f.argtypes = _ATTN_ARGS
+        L.blasst_decode_paged.restype = ctypes.c_int
+        L.blasst_decode_paged.argtypes = ([ctypes.c_void_p] * 7 + [ctypes.c_int] * 7 +
+                                          [ctypes.c_float, ctypes.c_float, ctypes.c_int] + [ctypes.c_void_p] * 3 +
+                                          [ctypes.POINTER(Opts)])
         L.blasst_calibrate_fit.restype = ctypes.c_int
         L.blasst_calibrate_fit.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
                                                                    ctypes.POINTER(ctypes.c_double)]
@@ -226,6 +230,54 @@ def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=No
                  want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hkv,
                  n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=dv)
     return o, lse, m, c
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, *, scale, lam=0.0, causal=False, num_splits=None,
+                 o=None, lse=None, skip_mask=True, skip_count=True, workspace=None, status_word=None, stream=None,
+                 seed_splits=False):
+    """Decode over a paged, ragged KV cache.
+
+    q [B,Hq,Lq,128]; k_pages/v_pages [num_pages, Hkv, 64, 128] bf16; block_table int32
+    [B, max_pages] (page of each 64-key block of each sequence); seq_lens int32 [B].
+    All CUDA tensors.  Returns (o, lse, skip_mask [B*Hkv, ceil(max_pages/32)] int32 or
+    None, skip_count [1] int64 or None).
+    """
+    import torch
+
+    for t, n in ((q, "q"), (k_pages, "k_pages"), (v_pages, "v_pages"), (block_table, "block_table"),
+                 (seq_lens, "seq_lens")):
+        _dev_tensor(t, n)
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    B, Hq, Lq, d = q.shape
+    num_pages, Hkv, page, dk = k_pages.shape
+    if page != 64 or dk != d or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("pages must be [num_pages, Hkv, 64, d] for both k and v")
+    if block_table.dim() != 2 or block_table.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("block_table [B, max_pages] and seq_lens [B] expected")
+    max_pages = block_table.shape[1]
+    if o is None:
+        o = torch.empty((B, Hq, Lq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    opts = Opts(num_splits=num_splits or 0, status_word=None if status_word is None else status_word.data_ptr(),
+                seed_splits=int(bool(seed_splits)))
+    if workspace is not None:
+        opts.workspace = workspace.data_ptr()
+        opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    dev = q.device
+    if skip_mask is True:
+        skip_mask = torch.empty((B * Hkv, mask_words(max_pages)), dtype=torch.int32, device=dev)
+    if skip_count is True:
+        skip_count = torch.empty(1, dtype=torch.int64, device=dev)
+    mask = skip_mask if isinstance(skip_mask, torch.Tensor) else None
+    count = skip_count if isinstance(skip_count, torch.Tensor) else None
+    rc = lib().blasst_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(o), _ptr(lse), _ptr(block_table), _ptr(seq_lens),
+        B, Hq, Hkv, Lq, max_pages, num_pages, d, float(scale), float(lam), int(bool(causal)),
+        _ptr(mask), _ptr(count), _stream(stream), ctypes.byref(opts))
+    _check(rc, "blasst_decode_paged")
+    return o, lse, mask, count
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

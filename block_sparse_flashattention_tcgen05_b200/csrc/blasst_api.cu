@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <climits>
 #include <cstring>
 #include <vector>
 
@@ -189,9 +190,18 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
 }
 
 // ------------------------------------------------------------------- decode
+// A paged KV cache: pages [num_pages, Hkv, 64, d]; sequence b has seq_lens[b] keys in
+// pages block_table[b * max_pages + i].  Both arrays are int32 in device memory.
+struct PagedCache {
+    const int *block_table;
+    const int *seq_lens;
+    int max_pages, num_pages;
+};
+
 blasst_status run_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                          int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
-                         unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib) {
+                         unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib,
+                         const PagedCache *pg = nullptr) {
     blasst_opts op = read_opts(opts_in);
     Common c;
     blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, op, &c);
@@ -204,6 +214,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     }
     if (op.block_n != 0 && op.block_n != kDecodeBlockN) return BLASST_ERR_UNSUPPORTED;
     if (op.seed_splits && d != 128) return BLASST_ERR_UNSUPPORTED;  // split seeding: GQA/MQA decode only
+    if (pg && (d != 128 || c.dv != 128 || c.krs != d || c.vrs != c.dv)) return BLASST_ERR_UNSUPPORTED;
     if (d == 576) return run_mla(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count,
                                  stream, op, c, calib);
     if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
@@ -225,11 +236,14 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     void *ws = op.workspace;
     if (!calib && ws && op.workspace_bytes < need) return BLASST_ERR_WORKSPACE;
 
+    // K/V: [planes, rows, d] with a plane per (sequence, KV head), or per (page, KV head)
+    const long long planes = pg ? (long long)pg->num_pages * Hkv : (long long)B * Hkv;
+    const long long plane_rows = pg ? kDecodeBlockN : Lk;
     CUtensorMap tk, tv;
-    st = make_tmap(&tk, k, d, Lk, (long long)B * Hkv, c.krs, 64, 64);
+    st = make_tmap(&tk, k, d, plane_rows, planes, c.krs, 64, 64);
     if (st != BLASST_OK) return st;
     if (!calib) {
-        st = make_tmap(&tv, v, c.dv, Lk, (long long)B * Hkv, c.vrs, 64, 64);
+        st = make_tmap(&tv, v, c.dv, plane_rows, planes, c.vrs, 64, 64);
         if (st != BLASST_OK) return st;
     } else {
         tv = tk;
@@ -269,6 +283,11 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     p.scale_log2 = (float)(scale * kLog2e);
     p.thr_log2 = log2_threshold(lambda);
     p.seed = op.seed_splits ? 1 : 0;
+    if (pg) {
+        p.block_table = pg->block_table;
+        p.seq_lens = pg->seq_lens;
+        p.num_pages = pg->num_pages;
+    }
     e = launch_decode(p, tk, tv, calib, R <= 8 ? 1 : 2, sm);
     if (e != cudaSuccess) return cuda_fail(e, "decode split kernel");
     if (!calib) {
@@ -364,6 +383,20 @@ blasst_status blasst_decode(const void *q, const void *k, const void *v, void *o
                             unsigned long long *skip_count, void *stream, const blasst_opts *opts) {
     return run_decode(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
                       opts, false);
+}
+
+blasst_status blasst_decode_paged(const void *q, const void *k_pages, const void *v_pages, void *o,
+                                 float *lse, const int *block_table, const int *seq_lens, int B, int Hq,
+                                             int Hkv, int Lq, int max_pages, int num_pages, int d, float scale,
+                                             float lambda, int causal, uint32_t *skip_mask,
+                                             unsigned long long *skip_count, void *stream, const blasst_opts *opts) {
+    if (!block_table || !seq_lens || !aligned(block_table, 4) || !aligned(seq_lens, 4)) return BLASST_ERR_INVALID;
+    if (max_pages <= 0 || num_pages <= 0) return BLASST_ERR_INVALID;
+    if ((long long)max_pages * kDecodeBlockN > INT_MAX || (long long)num_pages * (Hkv > 0 ? Hkv : 1) > INT_MAX)
+        return BLASST_ERR_INVALID;
+    const PagedCache pg{block_table, seq_lens, max_pages, num_pages};
+    return run_decode(q, k_pages, v_pages, o, lse, B, Hq, Hkv, Lq, max_pages * kDecodeBlockN, d, scale, lambda,
+                      causal, skip_mask, skip_count, stream, opts, false, &pg);
 }
 
 blasst_status blasst_calibrate(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,

@@ -39,6 +39,7 @@ constexpr int kThreads = kConsumerThreads + 64;
 constexpr int kStageBytes = kDecodeBlockN * 128 * 2;  // 64 keys x 128 dims bf16
 constexpr int kBoxBytes = kStageBytes / 2;             // 64 keys x 64 dims (one 128-byte swizzle box)
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadPage = 2;  // a page index or sequence length out of range
 
 struct DecodeSmemTail {
     uint64_t k_full[8];
@@ -63,6 +64,19 @@ __device__ __forceinline__ void set_timeout(DecodeSmemTail *t, unsigned int *sta
     if (status) atomicOr(status, kStatusTimeout);
 }
 
+// TMA coordinates (row, plane) of block blk of KV head hkv of sequence b.  A paged
+// cache maps the block through the block table; a page out of range is reported and
+// read as the plane past the end (the copy then fills zeros).
+__device__ __forceinline__ int2 kv_block_coord(const DecodeParams &p, int b, int hkv, int blk) {
+    if (!p.block_table) return make_int2(blk * kDecodeBlockN, b * p.Hkv + hkv);
+    int page = __ldg(p.block_table + (size_t)b * p.nb + blk);
+    if (page < 0 || page >= p.num_pages) {
+        if (p.status) atomicOr(p.status, kStatusBadPage);
+        page = p.num_pages;
+    }
+    return make_int2(0, page * p.Hkv + hkv);
+}
+
 template <int NT, int NK, int NV, bool CALIB>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -76,8 +90,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j0 = split * p.per_split;
-    const int j1 = min(p.nb, j0 + p.per_split);
+    // keys of this sequence: all Lk, or (paged) its own length, split the same way
+    int Lk = p.Lk, nbs = p.nb, per_split = p.per_split;
+    if (p.seq_lens) {
+        Lk = __ldg(p.seq_lens + b);
+        if (Lk < 0 || Lk > p.Lk) {
+            if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusBadPage);
+            Lk = min(max(Lk, 0), p.Lk);
+        }
+        nbs = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
+        per_split = (nbs + p.num_splits - 1) / p.num_splits;
+    }
+    const int j0 = split * per_split;
+    const int j1 = min(nbs, j0 + per_split);
     const int nblk = max(0, j1 - j0);
     const int bh = b * p.Hkv + hkv;
     // ring entries: [block 0 (seed)], then the split's blocks j0 .. j1-1
@@ -113,10 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const int blk = (seed && e == 0) ? 0 : j0 + e - seed;
+            const int2 cr = kv_block_coord(p, b, hkv, blk);
             uint8_t *dst = kring + slot * kStageBytes;
             mbar_arrive_expect_tx(&tl->k_full[slot], kStageBytes);
-            tma_load_3d(dst, &tmap_k, &tl->k_full[slot], 0, blk * kDecodeBlockN, bh);
-            tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, blk * kDecodeBlockN, bh);
+            tma_load_3d(dst, &tmap_k, &tl->k_full[slot], 0, cr.x, cr.y);
+            tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, cr.x, cr.y);
             issued++;
         }
         if (tl->abort) {  // let copies in flight land before the CTA exits
@@ -145,10 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 set_timeout(tl, p.status);
                 break;
             }
+            const int2 cr = kv_block_coord(p, b, hkv, j0 + jj);
             uint8_t *dst = vring + slot * kStageBytes;
             mbar_arrive_expect_tx(&tl->v_full[slot], kStageBytes);
-            tma_load_3d(dst, &tmap_v, &tl->v_full[slot], 0, (j0 + jj) * kDecodeBlockN, bh);
-            tma_load_3d(dst + kBoxBytes, &tmap_v, &tl->v_full[slot], 64, (j0 + jj) * kDecodeBlockN, bh);
+            tma_load_3d(dst, &tmap_v, &tl->v_full[slot], 0, cr.x, cr.y);
+            tma_load_3d(dst + kBoxBytes, &tmap_v, &tl->v_full[slot], 64, cr.x, cr.y);
             vk++;
         }
         if (tl->abort) {
@@ -182,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 2; e++) {
             const int c = nt * 8 + 2 * t4 + e;
             const int pos = c % p.Lq;
-            lastk[nt][e] = c >= p.R ? -1 : (p.causal ? pos + (p.Lk - p.Lq) : p.Lk - 1);
+            lastk[nt][e] = c >= p.R ? -1 : (p.causal ? pos + (Lk - p.Lq) : Lk - 1);
         }
 
     float Mall[NC];
@@ -243,8 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int nt = 0; nt < NT; nt++) {
 #pragma unroll
             for (int e = 0; e < 2; e++) {
-                s[nt][e] = key_lo <= lastk[nt][e] && key_lo < p.Lk ? acc[nt][e] * p.scale_log2 : NEG_INF;
-                s[nt][2 + e] = key_lo + 8 <= lastk[nt][e] && key_lo + 8 < p.Lk ? acc[nt][2 + e] * p.scale_log2 : NEG_INF;
+                s[nt][e] = key_lo <= lastk[nt][e] && key_lo < Lk ? acc[nt][e] * p.scale_log2 : NEG_INF;
+                s[nt][2 + e] = key_lo + 8 <= lastk[nt][e] && key_lo + 8 < Lk ? acc[nt][2 + e] * p.scale_log2 : NEG_INF;
                 float m = fmaxf(s[nt][e], s[nt][2 + e]);
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));

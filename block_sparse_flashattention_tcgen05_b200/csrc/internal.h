@@ -27,6 +27,11 @@ struct DecodeParams {
     float scale_log2;               // scale * log2(e)
     float thr_log2;                 // log2(lambda), -inf for lambda = 0
     int seed;                       // 1: splits after the first start from block 0's row maxima
+    // paged cache (null: contiguous): K/V pages [num_pages, Hkv, 64, 128]; sequence b has
+    // seq_lens[b] keys in pages block_table[b * nb + i]; Lk and nb are then the maxima
+    const int *block_table;
+    const int *seq_lens;
+    int num_pages;
 };
 
 struct CombineParams {

@@ -134,6 +134,34 @@ BLASST_API blasst_status blasst_decode(const void *q, const void *k, const void 
                             void *stream, const blasst_opts *opts);
 
 /*
+ * Decode over a paged, ragged KV cache.  Not on the pages as such: they report
+ * the method integrated into serving frameworks (xllm-io paper review,
+ * overview table; gist.science (de), section 1), whose caches are paged.  Per
+ * sequence the arithmetic is exactly blasst_decode's (same tile, 64-key blocks,
+ * num_splits chunks of that sequence's own blocks, lse combine, skip rule).
+ *
+ * k_pages, v_pages  [num_pages, Hkv, 64, d] bf16, dense: one 64-key page of one
+ *                   KV head is 64 x d contiguous elements.  d = dv = 128.
+ * block_table       device int32 [B, max_pages]: sequence b's block i lives in
+ *                   page block_table[b * max_pages + i].
+ * seq_lens          device int32 [B]: keys of sequence b, 0 .. max_pages * 64.
+ *                   Causal decode needs Lq <= seq_lens[b] (rows that see no key
+ *                   give O = 0 and lse = -inf).
+ * q, o, lse, skip_mask ([B, Hkv, W], W = ceil(max_pages / 32) words; blocks past
+ * a sequence's end are 0), skip_count, stream and opts (num_splits, workspace,
+ * status_word, seed_splits) as blasst_decode.  Argument errors return before
+ * any launch.  The device arrays are read by the kernel: a page index outside
+ * [0, num_pages) or a length outside [0, max_pages * 64] is not checked on the
+ * host; the kernel then reads zeros for that page (or clamps the length) and
+ * ORs 2 into *opts->status_word when given.
+ */
+BLASST_API blasst_status blasst_decode_paged(const void *q, const void *k_pages, const void *v_pages, void *o,
+                                             float *lse, const int *block_table, const int *seq_lens, int B, int Hq,
+                                             int Hkv, int Lq, int max_pages, int num_pages, int d, float scale,
+                                             float lambda, int causal, uint32_t *skip_mask,
+                                             unsigned long long *skip_count, void *stream, const blasst_opts *opts);
+
+/*
  * Calibration pass: the decision part of prefill (opts->mode = 0) or decode
  * (mode = 1) only -- QK^T, block row maxima, running max, gaps -- without
  * exp, P.V or V traffic.  v, o and lse may be NULL and are not touched.

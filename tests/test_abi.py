@@ -88,6 +88,28 @@ def test_split_seeding_only_on_gqa_decode(bl):
     assert _call(bl, "blasst_decode", d=576, opts=bl.Opts(seed_splits=1, dv=512)) == 2  # MLA
 
 
+def _paged(bl, **over):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, o=FAKE, lse=FAKE, table=FAKE, lens=FAKE, B=2, Hq=4, Hkv=1, Lq=1,
+             max_pages=8, num_pages=16, d=128, scale=0.088, lam=0.0, causal=0)
+    a.update(over)
+    return bl.lib().blasst_decode_paged(a["q"], a["kp"], a["vp"], a["o"], a["lse"], a["table"], a["lens"], a["B"],
+                                        a["Hq"], a["Hkv"], a["Lq"], a["max_pages"], a["num_pages"], a["d"],
+                                        a["scale"], a["lam"], a["causal"], None, None, None,
+                                        ctypes.byref(a.get("opts") or bl.Opts()))
+
+
+def test_paged_decode_arguments_rejected_before_launch(bl):
+    assert _paged(bl, table=None) == 1
+    assert _paged(bl, lens=None) == 1
+    assert _paged(bl, table=FAKE + 2) == 1                     # misaligned int32 array
+    assert _paged(bl, max_pages=0) == 1
+    assert _paged(bl, num_pages=0) == 1
+    assert _paged(bl, d=576) == 2                               # paged MLA cache: not built
+    assert _paged(bl, Hq=32) == 2                               # G * Lq > 16
+    assert _paged(bl, lam=1.0) == 1
+    assert _paged(bl, opts=bl.Opts(k_row_stride=256)) == 2      # pages are dense rows
+
+
 def test_calibrate_requires_gaps_and_valid_mode(bl):
     assert _call(bl, "blasst_calibrate") == 1                 # no gaps_out
     assert _call(bl, "blasst_calibrate", opts=bl.Opts(mode=7, gaps_out=FAKE)) == 1

@@ -176,7 +176,8 @@ def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o
            skip_mask=True, skip_count=True, workspace=None, status_word=None, stream=None, seed_splits=False):
     """Split-KV decode with block skipping.
 
-    GQA/MQA: q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA (16 splits by default).
+    GQA/MQA: q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA (16 splits by default);
+    (Hq/Hkv)*Lq <= 128 query rows per KV head.
     MLA: q [B,Hq,Lq,576], k [B,1,Lk,576], v = the same tensor as k, dv = 512 (V is
     the first 512 columns of each cache row; 2 splits by default).
     Returns (o, lse, skip_mask [B*Hkv, W] int32 or None, skip_count [1] int64 or None).

@@ -220,7 +220,10 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
     const int G = Hq / Hkv;
     const long long R = (long long)G * Lq;
-    if (R > 16) return BLASST_ERR_UNSUPPORTED;
+    // tiles of up to 16 rows: mma.sync kernel; 17..128 rows (MQA, large groups): tcgen05 kernel
+    const bool wide = R > 16;
+    if (R > 128) return BLASST_ERR_UNSUPPORTED;
+    if (wide && op.seed_splits) return BLASST_ERR_UNSUPPORTED;
     const int S = op.num_splits ? op.num_splits : 16;
     if (S < 1 || S > 65535) return BLASST_ERR_INVALID;
     if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;
@@ -247,6 +250,11 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         if (st != BLASST_OK) return st;
     } else {
         tv = tk;
+    }
+    CUtensorMap tq;  // wide tiles: q as [B][Hq*Lq][128], 128-row boxes
+    if (wide) {
+        st = make_tmap(&tq, q, d, (long long)Hq * Lq, B, d, 64, 128);
+        if (st != BLASST_OK) return st;
     }
 
     bool own_ws = false;
@@ -288,7 +296,11 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         p.seq_lens = pg->seq_lens;
         p.num_pages = pg->num_pages;
     }
-    e = launch_decode(p, tk, tv, calib, R <= 8 ? 1 : 2, sm);
+    if (wide) {
+        e = launch_decode_wide(p, tq, tk, tv, calib, sm);
+    } else {
+        e = launch_decode(p, tk, tv, calib, R <= 8 ? 1 : 2, sm);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "decode split kernel");
     if (!calib) {
         CombineParams cp;

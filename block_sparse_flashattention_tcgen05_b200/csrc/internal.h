@@ -82,6 +82,9 @@ void set_last_error(const char *msg);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
                           int nt, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t stream);
+// Decode tiles of 17..128 rows (d = 128) on tcgen05; tmap_q covers q as [B][Hq*Lq][128].
+cudaError_t launch_decode_wide(const DecodeParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                               const CUtensorMap &tmap_v, bool calib, cudaStream_t stream);
 cudaError_t launch_mla(const MlaParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k, bool calib,
                        cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,

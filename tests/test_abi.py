@@ -78,7 +78,8 @@ def test_invalid_arguments_rejected_before_launch(bl, fn):
 
 
 def test_decode_unsupported_tile_and_small_workspace(bl):
-    assert _call(bl, "blasst_decode", Hq=32, Hkv=1) == 2      # G * Lq > 16
+    assert _call(bl, "blasst_decode", Hq=256, Hkv=1) == 2     # G * Lq > 128
+    assert _call(bl, "blasst_decode", Hq=64, Hkv=1, opts=bl.Opts(seed_splits=1)) == 2  # seeding: tiles <= 16 rows
     assert _call(bl, "blasst_decode", opts=bl.Opts(workspace=FAKE, workspace_bytes=64)) == 3
     assert _call(bl, "blasst_decode", opts=bl.Opts(workspace=FAKE + 16, workspace_bytes=1 << 30)) == 1
 
@@ -105,7 +106,7 @@ def test_paged_decode_arguments_rejected_before_launch(bl):
     assert _paged(bl, max_pages=0) == 1
     assert _paged(bl, num_pages=0) == 1
     assert _paged(bl, d=576) == 2                               # paged MLA cache: not built
-    assert _paged(bl, Hq=32) == 2                               # G * Lq > 16
+    assert _paged(bl, Hq=256) == 2                              # G * Lq > 128
     assert _paged(bl, lam=1.0) == 1
     assert _paged(bl, opts=bl.Opts(k_row_stride=256)) == 2      # pages are dense rows
 

@@ -176,6 +176,61 @@ def test_decode_calibrate_matches_decode_masks(bl):
     assert np.max(np.abs(g[fin] - ref["gaps"][fin])) < 1e-3
 
 
+# ----------------------------------------------- wide tiles (17..128 rows, tcgen05)
+@pytest.mark.parametrize("lam", [0.0, 1e-3, 0.05, 0.5])
+@pytest.mark.parametrize("splits", [1, 4, 16])
+def test_decode_mqa_32_heads(bl, lam, splits):
+    inp = planted_decode(2, 32, 1, 64 * 41 + 13, 128, seed=51, reading="blk")
+    bits, _ = check_decode(bl, inp, lam, False, splits)
+    if lam == 0.0:
+        assert bits.sum() == 0
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.05])
+def test_decode_mqa_128_heads(bl, lam):
+    # every TMEM lane is a row
+    inp = planted_decode(2, 128, 1, 3000, 128, seed=52, reading="blk")
+    check_decode(bl, inp, lam, False, 4)
+
+
+def test_decode_gqa_group_32(bl):
+    inp = planted_decode(2, 64, 2, 2000, 128, seed=53, reading="blk")
+    check_decode(bl, inp, 0.05, False, 3)
+
+
+def test_decode_wide_causal_two_queries(bl):
+    inp = planted_decode(1, 64, 1, 2500, 128, Lq=2, seed=54, reading="blk")
+    check_decode(bl, inp, 0.1, True, 5)
+
+
+def test_decode_wide_short_cache_empty_splits(bl):
+    inp = planted_decode(2, 32, 1, 90, 128, seed=55, reading="lit")
+    check_decode(bl, inp, 0.3, False, 16)
+
+
+def test_decode_wide_calibrate_gaps(bl):
+    inp = planted_decode(2, 64, 2, 3000, 128, seed=56, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    gaps, mc, cc = bl.calibrate(q, k, scale=inp.scale, lam=0.05, mode="decode", num_splits=4)
+    _, _, md, cd = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=4)
+    torch.cuda.synchronize()
+    assert torch.equal(mc, md) and torch.equal(cc, cd)
+    ref = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.05, causal=False, is_decode=True,
+                           num_splits=4, BN=64)
+    g = gaps.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(ref["gaps"])
+    assert np.array_equal(np.isinf(g), np.isinf(ref["gaps"]))
+    assert np.max(np.abs(g[fin] - ref["gaps"][fin])) < 1e-3
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("lam", [0.0, 0.05])
+def test_decode_mqa_full_size_sampled(bl, lam):
+    # batch 8, 128 query heads on one KV head, 32768-key cache, 16 splits; oracle on sampled sequences
+    inp = planted_decode(8, 128, 1, 32768, 128, seed=57, reading="blk")
+    check_decode(bl, inp, lam, False, 16, tiles=[0, 5])
+
+
 # ------------------------------------------------------------- split seeding
 @pytest.mark.parametrize("lam", [0.0, 1e-3, 0.05, 0.5, 0.999])
 @pytest.mark.parametrize("splits", [4, 16])

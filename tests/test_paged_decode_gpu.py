@@ -110,6 +110,11 @@ def test_paged_seeded(bl, lam):
     check_paged(bl, inp, [4000, 1500, 333], lam, 8, seed_splits=True)
 
 
+def test_paged_mqa_wide_tile(bl):
+    inp = planted_decode(3, 64, 1, 2600, 128, seed=38, reading="blk")
+    check_paged(bl, inp, [2600, 65, 1300], 0.05, 4)
+
+
 def test_paged_single_key_sequences(bl):
     inp = planted_decode(3, 4, 1, 200, 128, seed=34, reading="lit")
     check_paged(bl, inp, [1, 63, 200], 0.3, 16)

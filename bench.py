@@ -47,6 +47,8 @@ PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, H
 DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk=32768, d=128, splits=16, seed=3)
 MLA = dict(workload="MLA decode, 128 heads, 576/512 latent, 32K cache, 2 splits", B=64, Hq=128, Lk=32768, splits=2,
            seed=5)
+MQA = dict(workload="decode MQA, 128 query heads on one KV head, 32K cache, 16 splits", B=64, Hq=128, Hkv=1,
+           Lk=32768, d=128, splits=16, seed=9)
 PREFILL_64K = dict(PREFILL, workload="prefill GQA 64K (Qwen3-8B-like attention shape)", L=65536, seed=4)
 QUICK_PREFILL = dict(PREFILL, workload="prefill GQA 4K (quick)", L=4096)
 QUICK_DECODE = dict(DECODE, workload="decode GQA 4K cache (quick)", B=4, Lk=4096)
@@ -303,6 +305,12 @@ class DecodeSeeded(Decode):
 
     kind = "decode_seeded"
     seed_splits = True
+
+
+class DecodeMqa(Decode):
+    """Decode with a 128-row tile (128 query heads on one KV head): the tcgen05 kernel."""
+
+    kind = "decode_mqa"
 
 
 class DecodePaged:
@@ -769,6 +777,7 @@ def main():
     ap.add_argument("--no-64k", action="store_true")
     ap.add_argument("--no-seeded", action="store_true", help="skip the split-seeded decode rows of the sweep")
     ap.add_argument("--no-paged", action="store_true", help="skip the paged, ragged decode rows of the sweep")
+    ap.add_argument("--no-mqa", action="store_true", help="skip the 128-head MQA decode rows of the sweep")
     ap.add_argument("--calibration", action="store_true",
                     help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
     args = ap.parse_args()
@@ -868,6 +877,9 @@ def main():
         if not args.no_paged:
             wls["decode_paged"] = DecodePaged(wls["decode"], dev,
                                               min_len=min(8192, wls["decode"].cfg["Lk"] // 4))
+        if not args.no_mqa:
+            mcfg_q = MQA if args.size == "full" else dict(MQA, B=max(2, MQA["B"] // 8), Lk=dcfg["Lk"])
+            wls["decode_mqa"] = DecodeMqa(mcfg_q, dev)
         if "mla" not in wls and not args.no_mla:
             wls["mla"] = Mla(mcfg, dev)
         if args.size == "full" and "prefill" in wls and not args.no_64k:

@@ -224,6 +224,9 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     const bool wide = R > 16;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
     if (wide && op.seed_splits) return BLASST_ERR_UNSUPPORTED;
+    if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + (op.num_splits ? op.num_splits : 16) - 1) /
+                        (op.num_splits ? op.num_splits : 16) > 1024)
+        return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 blocks per split
     const int S = op.num_splits ? op.num_splits : 16;
     if (S < 1 || S > 65535) return BLASST_ERR_INVALID;
     if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;

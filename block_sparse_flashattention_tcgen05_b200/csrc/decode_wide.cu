@@ -12,8 +12,9 @@
 // rescale, P = 2^(s - M_ref) in TMEM, O += P V_j (M = 128, N = 128, K = 64).
 //
 // Warp roles (224 threads): warps 0-3 softmax/decision (thread = row), warp 4 TMA
-// producer of Q (once) and K (4-stage ring), warp 5 TMEM allocation + tcgen05.mma
-// issue, warp 6 V producer (3-stage ring, kept blocks only).
+// producer of Q (once) and K (2-stage ring), warp 5 TMEM allocation + tcgen05.mma
+// issue, warp 6 V producer (2-stage ring, kept blocks only).  Two CTAs share an SM
+// (99 KB of shared memory and 256 TMEM columns each).
 // TMEM (256 columns): S [0,64), P [64,96) bf16, O [128,256).
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -31,7 +32,8 @@ constexpr int kBoxBytesQ = kRows * 128;    // 128 rows x 64 bf16
 constexpr int kBoxBytesKV = kBN * 128;     // 64 keys x 64 bf16
 constexpr int kStageBytes = 2 * kBoxBytesKV;
 constexpr int kQBytes = 2 * kBoxBytesQ;
-constexpr int kNK = 4, kNV = 3;
+constexpr int kNK = 2, kNV = 2;   // two CTAs per SM: each keeps two blocks of K and of V in flight
+constexpr int kMaxWideBlocks = 1024;  // blocks per split (decision array)
 constexpr uint32_t kColP = 64, kColO = 128;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kStatusTimeout = 1;
@@ -49,7 +51,7 @@ struct WideSmemTail {
 
 constexpr int wide_smem_bytes(bool calib) {
     return kQBytes + kNK * kStageBytes + (calib ? 0 : kNV * kStageBytes) + (int)sizeof(WideSmemTail) +
-           kMaxBlocksPerSplit + 1024;
+           kMaxWideBlocks + 1024;
 }
 
 __device__ __forceinline__ void set_timeout(WideSmemTail *t, unsigned int *status) {
@@ -69,7 +71,7 @@ __device__ __forceinline__ int2 block_coord(const DecodeParams &p, int b, int hk
 }
 
 template <bool CALIB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_wide_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
     extern __shared__ uint8_t smem_raw[];

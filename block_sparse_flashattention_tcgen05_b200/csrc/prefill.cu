@@ -57,7 +57,6 @@ struct PrefillSmemTail {
     uint64_t k_full[kStagesK], k_empty[kStagesK];
     uint64_t v_full[kStagesV], v_empty[kStagesV];
     uint64_t s_full[2], p_full[2], o_done[2];
-    uint64_t vote_bar[2];  // one arrival per softmax warp and block (blocks j >= 1)
     uint64_t mma_done;
     uint32_t tmem_base;
     int dec[2];
@@ -120,7 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tl->s_full[t], 1);
             mbar_init(&tl->p_full[t], kSoftmaxThreads / 32);
             mbar_init(&tl->o_done[t], 1);
-            mbar_init(&tl->vote_bar[t], kSoftmaxThreads / 32);
         }
         mbar_init(&tl->mma_done, 1);
         tl->abort = 0;
@@ -334,23 +332,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mn = fmaxf(m_true, mt);
             const bool vote = (mt == NEG_INF) || (mt - mn < p.thr_log2);
             // Tile-wide AND in two levels.  A warp with a row that forbids the skip
-            // knows the block is kept and goes on at once; only a warp whose rows all
-            // allow it waits for the other three warps' votes.  The first block is
-            // always kept and takes no vote.  (A warp reaches block j+1 only after all
-            // four warps published block j, so one barrier phase per block suffices.)
+            // knows the block is kept: it leaves its vote and arrives at the tile's named
+            // barrier without waiting.  Only warps whose rows all allow the skip wait
+            // there for the other three votes.  The first block is always kept and takes
+            // no vote.  (A warp reaches block j+1 only after all four warps published block
+            // j, so a barrier instance is complete before its id is used again; the ids
+            // also alternate with the block parity.)
             bool skip = false;
             if (j > 0) {
                 const bool wvote = __all_sync(0xffffffffu, vote);
                 uint8_t *vb = reinterpret_cast<uint8_t *>(&tl->votes[t][j & 1]);
-                if (lane == 0) {
-                    vb[wq] = wvote ? 1 : 0;
-                    mbar_arrive(&tl->vote_bar[t]);  // release: the vote byte is visible first
-                }
+                if (lane == 0) vb[wq] = wvote ? 1 : 0;
+                const int vid = 3 + 2 * t + (j & 1);
                 if (wvote) {
-                    if (mbar_wait(&tl->vote_bar[t], (j - 1) & 1, &tl->abort))
-                        skip = *reinterpret_cast<volatile uint32_t *>(vb) == 0x01010101u;
-                    else
-                        set_timeout(tl, p.status);
+                    bar_sync(vid, kSoftmaxThreads);
+                    skip = *reinterpret_cast<volatile uint32_t *>(vb) == 0x01010101u;
+                } else {
+                    bar_arrive(vid, kSoftmaxThreads);
                 }
             }
             if (CALIB && p.gaps) {

@@ -301,6 +301,13 @@ __device__ __forceinline__ bool bar_and(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
+// Count this warp's arrival at named barrier `id` (nthreads in all) without waiting;
+// the arriving threads' earlier memory accesses are visible to the threads that
+// complete the barrier with bar_sync.
+__device__ __forceinline__ void bar_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

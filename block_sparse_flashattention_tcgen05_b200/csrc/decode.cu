@@ -10,6 +10,9 @@
 //              N), block row maxima exchanged through shared memory, the
 //              tile-wide skip decision, then for kept blocks exp2 and
 //              O^T += V_j^T P^T (P re-laid out in registers with movmatrix).
+//              The exponentials and P.V of a block run DQ blocks after its
+//              decision (its scores wait in a register queue), so the V load
+//              that the decision starts overlaps the next blocks' S.
 //   warp 4     K producer: TMA loads of K blocks into a ring, as far ahead as
 //              the ring allows; K is read for every block.
 //   warp 5     V producer: waits for each block's published decision and
@@ -237,6 +240,103 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned long long n_skip = 0;
     const float NEG_INF = -CUDART_INF_F;
 
+    // Software pipeline: a block's decision is published (and its V load requested) DQ
+    // blocks before its exponentials and P.V run, so the V load is in flight meanwhile.
+    // The decided blocks wait in a small queue in registers (shifted statically).
+    constexpr int DQ = NT == 1 ? 2 : 1;
+    float qs[DQ][NT][4], qmo[DQ][NT][2], qmn[DQ][NT][2];
+    bool qk[DQ];
+#pragma unroll
+    for (int d = 0; d < DQ; d++) qk[d] = false;
+    // P.V of a kept block: rescale by the growth of the running max, P = 2^(s - M), O += P V
+    auto pv_block = [&](const float (&hs)[NT][4], const float (&hmo)[NT][2], const float (&hmn)[NT][2]) {
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+            float pv[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 2; e2++) {
+                const float mold = hmo[nt][e2], mnew = hmn[nt][e2];
+                const float alpha = (mnew == NEG_INF) ? 1.f : ex2(mold - mnew);
+                lsum[nt][e2] *= alpha;
+                lrnd[nt][e2] *= alpha;
+#pragma unroll
+                for (int mt = 0; mt < 8; mt++) {
+                    o_acc[mt][nt][e2] *= alpha;
+                    o_acc[mt][nt][2 + e2] *= alpha;
+                }
+                pv[e2] = hs[nt][e2] == NEG_INF ? 0.f : ex2(hs[nt][e2] - mnew);
+                pv[2 + e2] = hs[nt][2 + e2] == NEG_INF ? 0.f : ex2(hs[nt][2 + e2] - mnew);
+                lsum[nt][e2] += pv[e2] + pv[2 + e2];
+            }
+            const uint32_t lo = pack_bf16x2(pv[0], pv[1]);
+            const uint32_t hi = pack_bf16x2(pv[2], pv[3]);
+            lrnd[nt][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
+            lrnd[nt][1] += __uint_as_float(lo & 0xFFFF0000u) + __uint_as_float(hi & 0xFFFF0000u);
+            pb[nt][0] = movmatrix_t(lo);
+            pb[nt][1] = movmatrix_t(hi);
+        }
+        const int vslot = kept_count % NV;
+        if (!mbar_wait(&tl->v_full[vslot], (kept_count / NV) & 1, &tl->abort)) set_timeout(tl, p.status);
+        const uint8_t *vb = vring + vslot * kStageBytes;
+        {
+            const int mi = lane >> 3, ri = lane & 7;
+            const int key = warp * 16 + ri + 8 * (mi >> 1);
+#pragma unroll
+            for (int mt = 0; mt < 8; mt++) {
+                const int chunk = mt * 2 + (mi & 1);
+                uint32_t a[4];
+                ldsm_x4_t(smem_addr(vb + (chunk >> 3) * kBoxBytes + swz128(key, chunk & 7)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) mma_bf16_16816(o_acc[mt][nt], a, pb[nt]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl->v_empty[vslot]);
+        kept_count++;
+    };
+    // queue a decided block, and run P.V for the oldest one if it was kept
+    auto push_pop = [&](bool ck, const float (&cs)[NT][4], const float (&cmo)[NT][2], const float (&cmn)[NT][2]) {
+        const bool hk = qk[0];
+        float hs[NT][4], hmo[NT][2], hmn[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+            for (int i = 0; i < 4; i++) hs[nt][i] = qs[0][nt][i];
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                hmo[nt][i] = qmo[0][nt][i];
+                hmn[nt][i] = qmn[0][nt][i];
+            }
+        }
+#pragma unroll
+        for (int d = 0; d + 1 < DQ; d++) {
+            qk[d] = qk[d + 1];
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+                for (int i = 0; i < 4; i++) qs[d][nt][i] = qs[d + 1][nt][i];
+#pragma unroll
+                for (int i = 0; i < 2; i++) {
+                    qmo[d][nt][i] = qmo[d + 1][nt][i];
+                    qmn[d][nt][i] = qmn[d + 1][nt][i];
+                }
+            }
+        }
+        qk[DQ - 1] = ck;
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+            for (int i = 0; i < 4; i++) qs[DQ - 1][nt][i] = cs[nt][i];
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                qmo[DQ - 1][nt][i] = cmo[nt][i];
+                qmn[DQ - 1][nt][i] = cmn[nt][i];
+            }
+        }
+        if (hk) pv_block(hs, hmo, hmn);
+    };
+
     for (int e = 0; e < nent; e++) {
         const int jj = e - seed;  // block index within the split; -1: the seed block
         const int j = jj < 0 ? 0 : j0 + jj;
@@ -343,23 +443,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        if (CALIB) {
+        if constexpr (CALIB) {
             if (kept) {
 #pragma unroll
                 for (int c = 0; c < NC; c++) Mall[c] = Mn[c];
             }
-            continue;
-        }
-        if (!kept) continue;
-
-        // rescale by the growth of the running max, then P = 2^(s - M)
-        uint32_t pb[NT][2];
+        } else {
+        // queue the block: its scores and, for my columns, the running max before and after it
+        float cs[NT][4], cmo[NT][2], cmn[NT][2];
 #pragma unroll
-        for (int nt = 0; nt < NT; nt++) {
-            float pv[4];
+        for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-            for (int e = 0; e < 2; e++) {
-                const int c = nt * 8 + 2 * t4 + e;
+            for (int e2 = 0; e2 < 2; e2++) {
+                const int c = nt * 8 + 2 * t4 + e2;
                 float mold = NEG_INF, mnew = NEG_INF;
 #pragma unroll
                 for (int cc = 0; cc < NC; cc++)
@@ -367,46 +463,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mold = Mall[cc];
                         mnew = Mn[cc];
                     }
-                const float alpha = (mnew == NEG_INF) ? 1.f : ex2(mold - mnew);
-                lsum[nt][e] *= alpha;
-                lrnd[nt][e] *= alpha;
-#pragma unroll
-                for (int mt = 0; mt < 8; mt++) {
-                    o_acc[mt][nt][e] *= alpha;
-                    o_acc[mt][nt][2 + e] *= alpha;
-                }
-                pv[e] = s[nt][e] == NEG_INF ? 0.f : ex2(s[nt][e] - mnew);
-                pv[2 + e] = s[nt][2 + e] == NEG_INF ? 0.f : ex2(s[nt][2 + e] - mnew);
-                lsum[nt][e] += pv[e] + pv[2 + e];
+                cmo[nt][e2] = mold;
+                cmn[nt][e2] = mnew;
+                cs[nt][e2] = s[nt][e2];
+                cs[nt][2 + e2] = s[nt][2 + e2];
             }
-            const uint32_t lo = pack_bf16x2(pv[0], pv[1]);
-            const uint32_t hi = pack_bf16x2(pv[2], pv[3]);
-            lrnd[nt][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
-            lrnd[nt][1] += __uint_as_float(lo & 0xFFFF0000u) + __uint_as_float(hi & 0xFFFF0000u);
-            pb[nt][0] = movmatrix_t(lo);
-            pb[nt][1] = movmatrix_t(hi);
+        if (kept) {
+#pragma unroll
+            for (int c = 0; c < NC; c++) Mall[c] = Mn[c];
         }
-#pragma unroll
-        for (int c = 0; c < NC; c++) Mall[c] = Mn[c];
-
-        const int vslot = kept_count % NV;
-        if (!mbar_wait(&tl->v_full[vslot], (kept_count / NV) & 1, &tl->abort)) set_timeout(tl, p.status);
-        const uint8_t *vb = vring + vslot * kStageBytes;
-        {
-            const int mi = lane >> 3, ri = lane & 7;
-            const int key = warp * 16 + ri + 8 * (mi >> 1);
-#pragma unroll
-            for (int mt = 0; mt < 8; mt++) {
-                const int chunk = mt * 2 + (mi & 1);
-                uint32_t a[4];
-                ldsm_x4_t(smem_addr(vb + (chunk >> 3) * kBoxBytes + swz128(key, chunk & 7)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-                for (int nt = 0; nt < NT; nt++) mma_bf16_16816(o_acc[mt][nt], a, pb[nt]);
-            }
+        push_pop(kept, cs, cmo, cmn);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tl->v_empty[vslot]);
-        kept_count++;
+    }
+    if constexpr (!CALIB) {
+        // the last queued blocks
+        float zs[NT][4] = {}, zm[NT][2] = {};
+#pragma unroll
+        for (int d = 0; d < DQ; d++) push_pop(false, zs, zm, zm);
     }
 
     if (warp == 0 && lane == 0) {

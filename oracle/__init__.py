@@ -183,3 +183,84 @@ def threshold_for_sparsity(gaps, visited, target):
     lam = min(lam, np.nextafter(1.0, 0.0))
     achieved = float(np.count_nonzero(cand < math.log(lam))) / n_vis
     return lam, achieved
+
+
+def _as_f64(a):
+    """bf16 bit patterns (uint16) or real arrays -> float64."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def attention_backward(q, k, v, do, *, scale, causal, skip=None, BM=BM_PREFILL, BN=BN_PREFILL):
+    """Gradients of blocked attention with a FIXED skip mask (fp64, no blocking).
+
+    The forward is O = softmax_kept(scale * Q K^T) V, where a score (r, c)
+    takes part iff key c is visible to query r (c < Lk and, causal,
+    c <= r + Lk - Lq) and the (query tile r // BM, key block c // BN) pair is
+    not skipped; lse_r = log sum_kept exp(S_rc).  With the mask held constant
+    this is plain masked softmax attention, so its gradient is the textbook
+    one, written out step by step.  Skipped pairs carry P = 0 and so receive
+    no gradient, which is the optional sparsity-aware training the pages
+    describe (xllm-io paper review, section 3, "training procedure"):
+
+        P    = exp(S - lse) on kept entries, 0 elsewhere
+        dV   = P^T dO                  (summed over the query heads of a KV head)
+        dP   = dO V^T
+        D_r  = sum_c P_rc dP_rc
+        dS   = P * (dP - D)
+        dQ   = scale * dS K
+        dK   = scale * dS^T Q          (summed over the query heads of a KV head)
+
+    q [B, Hq, Lq, d], k [B, Hkv, Lk, d], v [B, Hkv, Lk, dv], do [B, Hq, Lq, dv]:
+    uint16 bf16 bit patterns or real arrays.  skip: None (nothing skipped) or
+    uint8 [B * Hq * ceil(Lq / BM), ceil(Lk / BN)], 1 = skipped, tiles ordered
+    (b, hq, query tile) -- the prefill mask layout.  A row with no kept score
+    has O = 0, lse = -inf and no gradient.
+    Returns dict dq, dk, dv, o (float64) and lse (float64, natural log).
+    """
+    Q, K, V, dO = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    dv = V.shape[3]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    nq = (Lq + BM - 1) // BM
+    nb = (Lk + BN - 1) // BN
+    if skip is not None:
+        skip = np.asarray(skip, dtype=np.uint8).reshape(B, Hq, nq, nb)
+    rows = np.arange(Lq)[:, None]
+    cols = np.arange(Lk)[None, :]
+    visible = np.ones((Lq, Lk), bool)
+    if causal:
+        visible &= cols <= rows + (Lk - Lq)
+    dq = np.zeros((B, Hq, Lq, d))
+    dk = np.zeros((B, Hkv, Lk, d))
+    dvv = np.zeros((B, Hkv, Lk, dv))
+    o = np.zeros((B, Hq, Lq, dv))
+    lse = np.full((B, Hq, Lq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            keep = visible.copy()
+            if skip is not None:
+                keep &= ~skip[b, h][rows // BM, cols // BN].astype(bool)
+            S = scale * (Q[b, h] @ K[b, hk].T)
+            Sm = np.where(keep, S, -np.inf)
+            m = Sm.max(axis=1, keepdims=True)
+            has = np.isfinite(m[:, 0])
+            m = np.where(np.isfinite(m), m, 0.0)
+            E = np.where(keep, np.exp(Sm - m), 0.0)
+            ell = E.sum(axis=1, keepdims=True)
+            P = np.divide(E, ell, out=np.zeros_like(E), where=ell > 0)
+            lse[b, h] = np.where(has, m[:, 0] + np.log(np.where(has, ell[:, 0], 1.0)), -np.inf)
+            o[b, h] = P @ V[b, hk]
+            dvv[b, hk] += P.T @ dO[b, h]
+            dP = dO[b, h] @ V[b, hk].T
+            D = (P * dP).sum(axis=1, keepdims=True)
+            dS = P * (dP - D)
+            dq[b, h] = scale * (dS @ K[b, hk])
+            dk[b, hk] += scale * (dS.T @ Q[b, h])
+    return dict(dq=dq, dk=dk, dv=dvv, o=o, lse=lse)

@@ -238,6 +238,55 @@ class Prefill:
         hl.copy_(self.lse, non_blocking=True)
 
 
+class Backward(Prefill):
+    """Fixed-mask backward on the prefill workload's shape: the forward at a given
+    lambda supplies o, lse and the skip mask (untimed: it runs in the warm-up call
+    whenever lambda or the skip counter changes); the timed call is the backward
+    alone (prep, main kernel, dq finalize).  Work: the five 128x128x128 products
+    of every kept pair (S, dP, dQ, dV, dK)."""
+    kind = "backward"
+
+    def __init__(self, cfg, device, fwd=None):
+        import torch
+
+        if fwd is not None:  # share the forward workload's inputs
+            self.__dict__.update({k: v for k, v in fwd.__dict__.items() if k not in ("o", "lse")})
+        else:
+            super().__init__(cfg, device)
+        import synth
+
+        c = self.cfg
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:3], dtype=torch.float32, device=device)
+        self.dout = to_dev(synth.upstream_grad(c["B"], c["Hq"], c["L"], c["d"], seed=c["seed"]), device)
+        self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        self.ws = torch.empty(self.bl.backward_workspace_bytes(c["B"], c["Hq"], c["L"]), dtype=torch.uint8,
+                              device=device)
+        nq = (c["L"] + 127) // 128
+        self.mask = torch.zeros((c["B"] * c["Hq"] * nq, self.bl.mask_words(nq)), dtype=torch.int32, device=device)
+        self._fwd_key = None
+        self.launches = 3
+
+    def forward(self, lam):
+        self.bl.prefill(self.q, self.k, self.v, scale=self.inp.scale, lam=lam, causal=True, o=self.o, lse=self.lse,
+                        skip_mask=self.mask, skip_count=self.count)
+        self._fwd_key = (lam, id(self.count))
+
+    def call(self, lam, stream=None):
+        if self._fwd_key != (lam, id(self.count)):
+            self.forward(lam)
+        return self.bl.prefill_backward(self.q, self.k, self.v, self.o, self.lse, self.dout, scale=self.inp.scale,
+                                        causal=True, skip_mask=self.mask, dq=self.dq, dk=self.dk, dv=self.dv,
+                                        workspace=self.ws, stream=stream)
+
+    def work(self, skipped):
+        return 5 * FLOP_PER_PAIR * (self.visited - skipped)
+
+    def host_bytes(self):
+        return (self.inp.q.nbytes * 3 + self.inp.k.nbytes + self.inp.v.nbytes + self.lse.numel() * 4,
+                self.inp.q.nbytes + self.inp.k.nbytes * 2)
+
+
 class Decode:
     kind = "decode"
     unit = "GB/s"
@@ -597,6 +646,8 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
 
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     rng = np.random.default_rng(seed_tiles)
+    if wl_kind == "backward":
+        return oracle_backward_sample(cfg, lam_target, budget_s, seed_tiles)
     if wl_kind == "prefill":
         c = cfg
         inp = synth.planted_prefill(c["B"], c["Hq"], c["Hkv"], c["L"], c["d"], seed=c["seed"], reading="blk")
@@ -652,6 +703,44 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
                        f"({'last quarter of the sequence' if wl_kind == 'prefill' else 'whole KV heads'}), "
                        f"lambda={lam:.4g} for ~{lam_target:.0%} sparsity on the sample, {dt:.1f} s",
                 seconds=dt)
+
+
+def oracle_backward_sample(cfg, lam_target=0.75, budget_s=10.0, seed=0):
+    """Time the fp64 backward oracle (as it stands) on a bounded sample of the
+    backward workload: the first Ls tokens of one KV head's query-head group
+    (the oracle forms the whole Ls x Ls score matrix), its forward mask from the
+    C oracle at a lambda for ~lam_target sparsity.  Ls doubles until the budget."""
+    import numpy as np
+
+    import oracle
+    import synth
+
+    c = cfg
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    G = c["Hq"] // c["Hkv"]
+    kv = seed % c["Hkv"]
+    inp = synth.planted_prefill(1, c["Hq"], c["Hkv"], min(c["L"], 8192), c["d"], seed=c["seed"], reading="blk")
+    do = synth.upstream_grad(1, c["Hq"], min(c["L"], 8192), c["d"], seed=c["seed"])
+    Ls, dt, res = 1024, 0.0, None
+    while True:
+        q = np.ascontiguousarray(inp.q[:, kv * G:(kv + 1) * G, :Ls])
+        k = np.ascontiguousarray(inp.k[:, kv:kv + 1, :Ls])
+        v = np.ascontiguousarray(inp.v[:, kv:kv + 1, :Ls])
+        d_o = np.ascontiguousarray(do[:, kv * G:(kv + 1) * G, :Ls])
+        f0 = oracle.attention(q, k, v, scale=inp.scale, lam=0.0, causal=True)
+        lam, _ = oracle.threshold_for_sparsity(f0["gaps"], f0["visited"], lam_target)
+        f = oracle.attention(q, k, v, scale=inp.scale, lam=lam, causal=True)
+        t0 = time.time()
+        oracle.attention_backward(q, k, v, d_o, scale=inp.scale, causal=True, skip=f["skip"])
+        dt = time.time() - t0
+        res = (Ls, lam, f["n_visited"] - f["n_skipped"], f["n_skipped"] / max(1, f["n_visited"]))
+        if dt * 4.5 > budget_s or Ls * 2 > min(c["L"], 8192):
+            break
+        Ls *= 2
+    Ls, lam, kept, sp = res
+    return dict(value=5 * FLOP_PER_PAIR * kept / dt / 1e12, unit="TFLOP/s", cores=cores, kind="oracle",
+                sample=f"first {Ls} tokens of KV head {kv}'s {G} query heads, lambda={lam:.4g} "
+                       f"({sp:.0%} of pairs skipped), {dt:.1f} s", seconds=dt)
 
 
 def oracle_mha1024(lam_a=32.0, budget_s=3.0):
@@ -736,7 +825,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     wl_kind = args.workload
-    cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2}[wl_kind]]
+    cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2, "backward": 0}[wl_kind]]
     per_step = []
     vals = []
     budget = float(os.environ.get("BLASST_REF_STEP_SECONDS", "8"))
@@ -767,7 +856,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--workload", choices=["prefill", "decode", "mla"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "decode", "mla", "backward"], default="prefill")
     ap.add_argument("--size", choices=sorted(SIZES), default="full",
                     help="full = the benchmark shapes; medium = profiling size; quick = smoke-testing the bench")
     ap.add_argument("--no-sweep", action="store_true")
@@ -778,6 +867,7 @@ def main():
     ap.add_argument("--no-seeded", action="store_true", help="skip the split-seeded decode rows of the sweep")
     ap.add_argument("--no-paged", action="store_true", help="skip the paged, ragged decode rows of the sweep")
     ap.add_argument("--no-mqa", action="store_true", help="skip the 128-head MQA decode rows of the sweep")
+    ap.add_argument("--no-backward", action="store_true", help="skip the fixed-mask backward rows of the sweep")
     ap.add_argument("--calibration", action="store_true",
                     help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
     args = ap.parse_args()
@@ -820,6 +910,9 @@ def main():
         wls["decode"] = Decode(dcfg, dev)
     if headline_kind == "mla":
         wls["mla"] = Mla(mcfg, dev)
+    if headline_kind == "backward":
+        wls["backward"] = Backward(pcfg, dev)
+        wls["backward"].count = torch.zeros(1, dtype=torch.int64, device=dev)
     # the headline workload is calibrated and timed before any other workload runs
     lams = {headline_kind: lambdas_for_targets(wls[headline_kind], wls[headline_kind].calibrate())}
 
@@ -882,8 +975,12 @@ def main():
             wls["decode_mqa"] = DecodeMqa(mcfg_q, dev)
         if "mla" not in wls and not args.no_mla:
             wls["mla"] = Mla(mcfg, dev)
+        if "prefill" in wls and "backward" not in wls and not args.no_backward:
+            wls["backward"] = Backward(pcfg, dev, fwd=wls["prefill"])
         if args.size == "full" and "prefill" in wls and not args.no_64k:
             wls["prefill_64k"] = Prefill(PREFILL_64K, dev)
+        if "backward" in wls and "prefill" in lams and "backward" not in lams:
+            lams["backward"] = lams["prefill"]  # same inputs, same forward masks
         for k, w in wls.items():
             if k not in lams:
                 lams[k] = w.lambdas() if hasattr(w, "lambdas") else lambdas_for_targets(w, w.calibrate())

@@ -12,7 +12,8 @@ import os
 
 __all__ = [
     "BlasstError", "lib", "prefill", "decode", "decode_noalloc", "calibrate", "calibrate_fit", "calibrate_threshold",
-    "visited_pairs", "decode_workspace_bytes", "mask_words", "Opts", "STATUS",
+    "visited_pairs", "decode_workspace_bytes", "mask_words", "Opts", "STATUS", "prefill_backward",
+    "backward_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +81,12 @@ def lib() -> ctypes.CDLL:
         L.blasst_decode_paged.argtypes = ([ctypes.c_void_p] * 7 + [ctypes.c_int] * 7 +
                                           [ctypes.c_float, ctypes.c_float, ctypes.c_int] + [ctypes.c_void_p] * 3 +
                                           [ctypes.POINTER(Opts)])
+        L.blasst_prefill_backward.restype = ctypes.c_int
+        L.blasst_prefill_backward.argtypes = ([ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 +
+                                              [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.POINTER(Opts)])
+        L.blasst_backward_workspace_bytes.restype = ctypes.c_size_t
+        L.blasst_backward_workspace_bytes.argtypes = [ctypes.c_int] * 3
         L.blasst_calibrate_fit.restype = ctypes.c_int
         L.blasst_calibrate_fit.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
                                                                    ctypes.POINTER(ctypes.c_double)]
@@ -170,6 +177,41 @@ def prefill(q, k, v, *, scale, lam=0.0, causal=True, o=None, lse=None, skip_mask
                  want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hq * nq,
                  n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=d)
     return o, lse, m, c
+
+
+def prefill_backward(q, k, v, o, lse, dout, *, scale, causal=True, skip_mask=None, dq=None, dk=None, dv=None,
+                     workspace=None, status_word=None, stream=None):
+    """Gradients (dq, dk, dv) of prefill attention with the forward's skip mask held fixed.
+
+    q, k, v, o, lse: the forward's tensors; dout [B,Hq,Lq,128] bf16, the gradient of o;
+    skip_mask: the forward's mask (int32 [B*Hq*ceil(Lq/128), W]) or None (nothing skipped).
+    Returns bf16 dq [B,Hq,Lq,128], dk, dv [B,Hkv,Lk,128].
+    """
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout")):
+        _dev_tensor(t, n)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if dq is None:
+        dq = torch.empty_like(q)
+    if dk is None:
+        dk = torch.empty_like(k)
+    if dv is None:
+        dv = torch.empty_like(v)
+    opts = Opts(status_word=None if status_word is None else status_word.data_ptr())
+    if workspace is not None:
+        opts.workspace = workspace.data_ptr()
+        opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().blasst_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                       _ptr(dv), B, Hq, Hkv, Lq, Lk, d, float(scale), int(bool(causal)),
+                                       _ptr(skip_mask), _stream(stream), ctypes.byref(opts))
+    _check(rc, "blasst_prefill_backward")
+    return dq, dk, dv
+
+
+def backward_workspace_bytes(B, Hq, Lq) -> int:
+    return int(lib().blasst_backward_workspace_bytes(B, Hq, Lq))
 
 
 def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o=None, lse=None,

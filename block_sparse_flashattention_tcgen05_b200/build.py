@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libblasst.so")
-SOURCES = ["blasst_api.cu", "decode.cu", "decode_wide.cu", "prefill.cu", "mla.cu", "decode_noalloc.cu"]
+SOURCES = ["blasst_api.cu", "decode.cu", "decode_wide.cu", "prefill.cu", "mla.cu", "decode_noalloc.cu", "backward.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 

@@ -1,0 +1,507 @@
+// backward.cu -- attention backward for the prefill tiling with the forward's
+// skip mask held fixed: skipped (query tile, KV block) pairs get no gradient,
+// which is the optional sparsity-aware training of the pages (xllm-io paper
+// review, section 3, "training procedure": the forward skips blocks, the
+// skipped blocks receive no gradient in the backward pass).
+//
+// Three launches:
+//   prep      per query row: delta = rowsum(dO * O) (fp32), lse2 = lse*log2(e)
+//             (+inf on padding rows and rows that saw no key, so their P is 0),
+//             and the row of the fp32 dQ accumulator set to zero;
+//   main      one CTA per (KV block j of 128 keys, KV head, sequence) walks the
+//             kept (query tile i, query head) pairs of its KV head in order
+//             and accumulates dK_j and dV_j over all of them in tensor memory;
+//             dQ_i contributions go to the fp32 accumulator by coalesced
+//             red.add (each warp adds 128 contiguous bytes of one query row);
+//   finalize  dQ accumulator -> bf16 dq.
+//
+// Main kernel, per pair (S^T etc. are key-major: TMEM lane = key of block j):
+//   S^T  = K_j Q_i^T                        tcgen05, A = K (K-major), B = Q (K-major)
+//   dP^T = V_j dO_i^T                       tcgen05, A = V, B = dO (both K-major)
+//   P^T  = 2^(S^T * scale*log2e - lse2)     masked (key >= Lk, causal) to 0
+//   dS^T = scale * P^T (dP^T - delta)       bf16 into shared memory
+//   dQ^T = K_j^T dS^T                       A = K (MN-major), B = dS^T (MN-major)
+//   dV  += P^T dO_i                         A = P^T from TMEM (bf16), B = dO (MN-major)
+//   dK  += dS^T Q_i                         A = dS^T (K-major), B = Q (MN-major)
+//
+// Warp roles (320 threads):
+//   warps 0-7  compute: warp w owns TMEM lanes 32*(w%4).. (keys for S^T/dP^T,
+//              head dims for dQ^T) and query half w/4 (64 columns);
+//   warp 8     TMA producer: K_j, V_j once; Q_i, dO_i, lse2_i, delta_i per pair
+//              into a 2-stage ring;
+//   warp 9     allocates TMEM and issues every tcgen05.mma from one thread.
+//
+// TMEM (512 columns): S^T [0,128) -> P^T (bf16; queries 0-63 in [0,32),
+// 64-127 in [64,96)); dP^T [128,256) -> dQ^T; dV [256,384); dK [384,512).
+//
+// MMA issue order per pair t: dP(t) [after the dQ^T(t-1) columns are read],
+// then, once dS^T(t) is ready: dQ^T(t), dV(t), S(t+1), dK(t).  The compute
+// warps form P(t+1) from S(t+1) while dK(t) and dP(t+1) run.  Operations
+// issued by one thread execute in issue order, so S(t+1) overwrites P^T(t)
+// only after dV(t) has read it, and a commit covers every earlier operation.
+#include <climits>
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace blasst {
+namespace {
+
+constexpr int kComputeWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
+constexpr int kBoxBytes = kTileBytes / 2;  // 128 rows x 64 bf16 (one 128-byte swizzle box)
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusSmemAlign = 4;
+
+struct BwdTail {
+    float lse2[2][128];   // per stage: lse * log2(e) of the pair's 128 query rows
+    float delta[2][128];  // per stage: rowsum(dO * O)
+    uint64_t kv_full;
+    uint64_t qdo_full[2], qdo_empty[2];
+    uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// K_j, V_j, Q/dO stages, dS^T; the base is 1024-byte aligned (checked)
+constexpr int kSmemBytes = 7 * kTileBytes + (int)sizeof(BwdTail);
+
+__device__ __forceinline__ void set_timeout(BwdTail *t, unsigned int *status) {
+    t->abort = 1;
+    if (status) atomicOr(status, kStatusTimeout);
+}
+
+// First query tile whose rows see a key of block j (tiles before it are not
+// visited by the forward for this block).
+__device__ __forceinline__ int first_tile(const BwdParams &p, int j) {
+    if (!p.causal) return 0;
+    const int need = j * 128 - (p.Lk - p.Lq) - 127;  // tile i qualifies iff i*128 >= need
+    return need <= 0 ? 0 : (need + 127) / 128;
+}
+
+// From (i, g) inclusive, move to the next pair (tile i, head g of the group)
+// that the forward kept for block j.  False when none is left.
+__device__ __forceinline__ bool next_pair(const BwdParams &p, int b, int hkv, int j, int &i, int &g) {
+    while (i < p.nq) {
+        if (!p.skip_mask) return true;
+        const int hq = hkv * p.G + g;
+        const uint32_t w = __ldg(p.skip_mask + (((size_t)b * p.Hq + hq) * p.nq + i) * p.words + (j >> 5));
+        if (!((w >> (j & 31)) & 1u)) return true;
+        if (++g == p.G) {
+            g = 0;
+            ++i;
+        }
+    }
+    return false;
+}
+
+// Bounded wait whose outcome is the same on every lane of the warp: the compute
+// warps issue warp-collective TMEM loads and stores after their waits, so a lane
+// must never leave a loop that the rest of its warp stays in.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+__device__ __forceinline__ void advance(const BwdParams &p, int &i, int &g) {
+    if (++g == p.G) {
+        g = 0;
+        ++i;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const BwdParams p, const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_do,
+               const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_addr(smem) & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusSmemAlign);
+        return;
+    }
+    uint8_t *sK = smem;
+    uint8_t *sV = smem + kTileBytes;
+    uint8_t *sQ = smem + 2 * kTileBytes;   // 2 stages
+    uint8_t *sdO = smem + 4 * kTileBytes;  // 2 stages
+    uint8_t *sdS = smem + 6 * kTileBytes;  // dS^T: [128 keys][128 queries] as two 64-query boxes
+    BwdTail *tl = reinterpret_cast<BwdTail *>(smem + 7 * kTileBytes);
+
+    // blocks with more query tiles first (causal: small j has the most pairs)
+    const int j = blockIdx.x / p.Hkv;
+    const int hkv = blockIdx.x % p.Hkv;
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kvrow = b * p.Hkv + hkv;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&tl->kv_full, 1);
+        for (int s = 0; s < 2; s++) {
+            mbar_init(&tl->qdo_full[s], 1);
+            mbar_init(&tl->qdo_empty[s], 1);
+        }
+        mbar_init(&tl->s_full, 1);
+        mbar_init(&tl->dp_full, 1);
+        mbar_init(&tl->ds_ready, kComputeWarps);
+        mbar_init(&tl->dq_full, 1);
+        mbar_init(&tl->dq_free, kComputeWarps);
+        mbar_init(&tl->acc_done, 1);
+        tl->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&tl->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tl->tmem_base;
+    int n_steps = 0;  // pairs processed (compute warps: for the epilogue)
+
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_do);
+            tma_prefetch_desc(&tmap_k);
+            tma_prefetch_desc(&tmap_v);
+            mbar_arrive_expect_tx(&tl->kv_full, 2 * kTileBytes);
+            tma_load_3d(sK, &tmap_k, &tl->kv_full, 0, j * 128, kvrow);
+            tma_load_3d(sK + kBoxBytes, &tmap_k, &tl->kv_full, 64, j * 128, kvrow);
+            tma_load_3d(sV, &tmap_v, &tl->kv_full, 0, j * 128, kvrow);
+            tma_load_3d(sV + kBoxBytes, &tmap_v, &tl->kv_full, 64, j * 128, kvrow);
+            int i = first_tile(p, j), g = 0, t = 0;
+            while (!tl->abort && next_pair(p, b, hkv, j, i, g)) {
+                const int st = t & 1;
+                if (t >= 2 && !mbar_wait(&tl->qdo_empty[st], ((t >> 1) & 1) ^ 1, &tl->abort)) {
+                    set_timeout(tl, p.status);
+                    break;
+                }
+                const int qrow = b * p.Hq + hkv * p.G + g;
+                const size_t rbase = (size_t)qrow * p.Lq_pad + (size_t)i * 128;
+                mbar_arrive_expect_tx(&tl->qdo_full[st], 2 * kTileBytes + 2 * 512);
+                uint8_t *q_dst = sQ + st * kTileBytes;
+                uint8_t *do_dst = sdO + st * kTileBytes;
+                tma_load_3d(q_dst, &tmap_q, &tl->qdo_full[st], 0, i * 128, qrow);
+                tma_load_3d(q_dst + kBoxBytes, &tmap_q, &tl->qdo_full[st], 64, i * 128, qrow);
+                tma_load_3d(do_dst, &tmap_do, &tl->qdo_full[st], 0, i * 128, qrow);
+                tma_load_3d(do_dst + kBoxBytes, &tmap_do, &tl->qdo_full[st], 64, i * 128, qrow);
+                bulk_load(&tl->lse2[st][0], p.lse2 + rbase, 512, &tl->qdo_full[st]);
+                bulk_load(&tl->delta[st][0], p.delta + rbase, 512, &tl->qdo_full[st]);
+                t++;
+                advance(p, i, g);
+            }
+            // loads nobody will wait for (after an abort) land before the CTA exits
+            mbar_wait(&tl->kv_full, 0, nullptr);
+            if (tl->abort)
+                for (int u = max(0, t - 2); u < t; u++) mbar_wait(&tl->qdo_full[u & 1], (u >> 1) & 1, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t dhi = umma_desc_hi_sw128();
+            constexpr uint32_t idesc_kk = umma_idesc_bf16_mn(128, 128, 0, 0);  // S^T, dP^T
+            constexpr uint32_t idesc_kmn = umma_idesc_bf16_mn(128, 128, 0, 1); // dV (A in TMEM), dK
+            constexpr uint32_t idesc_mnmn = umma_idesc_bf16_mn(128, 128, 1, 1);  // dQ^T
+            // K-major operands: 16-wide K steps inside a 64-wide swizzle box, then the next box
+            const uint32_t k_km = umma_desc_lo(smem_addr(sK), 16);
+            const uint32_t v_km = umma_desc_lo(smem_addr(sV), 16);
+            const uint32_t q_km = umma_desc_lo(smem_addr(sQ), 16);
+            const uint32_t do_km = umma_desc_lo(smem_addr(sdO), 16);
+            const uint32_t ds_km = umma_desc_lo(smem_addr(sdS), 16);
+            // MN-major operands: the two 64-wide MN boxes are kBoxBytes apart; a K step is 16 rows
+            const uint32_t k_mn = umma_desc_lo(smem_addr(sK), kBoxBytes);
+            const uint32_t q_mn = umma_desc_lo(smem_addr(sQ), kBoxBytes);
+            const uint32_t do_mn = umma_desc_lo(smem_addr(sdO), kBoxBytes);
+            const uint32_t ds_mn = umma_desc_lo(smem_addr(sdS), kBoxBytes);
+            constexpr uint32_t kStage16 = kTileBytes >> 4;
+            auto koff = [](int kk) { return (uint32_t)((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4; };
+            auto issue_s = [&](int st) {  // S^T = K Q^T into [0,128)
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ss2(tmem, k_km + koff(kk), q_km + st * kStage16 + koff(kk), dhi, idesc_kk, kk > 0);
+            };
+            bool ok = mbar_wait(&tl->kv_full, 0, &tl->abort);
+            int i = first_tile(p, j), g = 0, t = 0;
+            bool have = ok && next_pair(p, b, hkv, j, i, g);
+            if (have) {
+                if (!mbar_wait(&tl->qdo_full[0], 0, &tl->abort)) {
+                    set_timeout(tl, p.status);
+                    have = false;
+                } else {
+                    tc_fence_after();
+                    issue_s(0);
+                    umma_commit(&tl->s_full);
+                }
+            }
+            while (have) {
+                const int st = t & 1;
+                // dP^T(t) = V dO^T into [128,256), once dQ^T(t-1) has been read out
+                if (t > 0 && !mbar_wait(&tl->dq_free, (t - 1) & 1, &tl->abort)) {
+                    set_timeout(tl, p.status);
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ss2(tmem + 128, v_km + koff(kk), do_km + st * kStage16 + koff(kk), dhi, idesc_kk, kk > 0);
+                umma_commit(&tl->dp_full);
+                if (!mbar_wait(&tl->ds_ready, t & 1, &tl->abort)) {
+                    set_timeout(tl, p.status);
+                    break;
+                }
+                tc_fence_after();
+                // dQ^T = K^T dS^T (K = 128 keys) into [128,256)
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ss2(tmem + 128, k_mn + kk * (2048 >> 4), ds_mn + kk * (2048 >> 4), dhi, idesc_mnmn, kk > 0);
+                umma_commit(&tl->dq_full);
+                // dV += P^T dO (K = 128 queries; P^T halves at TMEM columns 0 and 64)
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ts2(tmem + 256, tmem + (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8),
+                             do_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn, (t > 0 || kk > 0) ? 1u : 0u);
+                // next pair's S^T, so that its softmax overlaps dK(t) and dP(t+1)
+                int ni = i, ng = g;
+                advance(p, ni, ng);
+                const bool more = next_pair(p, b, hkv, j, ni, ng);
+                if (more) {
+                    const int nst = (t + 1) & 1;
+                    if (!mbar_wait(&tl->qdo_full[nst], ((t + 1) >> 1) & 1, &tl->abort)) {
+                        set_timeout(tl, p.status);
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_s(nst);
+                    umma_commit(&tl->s_full);
+                }
+                // dK += dS^T Q (K = 128 queries)
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ss2(tmem + 384, ds_km + koff(kk), q_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn,
+                             (t > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&tl->qdo_empty[st]);
+                t++;
+                i = ni;
+                g = ng;
+                have = more;
+            }
+            // every MMA of this thread has completed: dK, dV final, TMEM free to release
+            umma_commit(&tl->acc_done);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ compute warps
+        const int wq = warp & 3;   // TMEM lane quadrant
+        const int hh = warp >> 2;  // query half: columns 64*hh .. 64*hh+63
+        const int r = wq * 32 + lane;  // key row within the block (S^T, dP^T), head dim (dQ^T)
+        const int key = j * 128 + r;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const int shift = p.Lk - p.Lq;
+        int i = first_tile(p, j), g = 0, t = 0;
+        while (__all_sync(0xffffffffu, !tl->abort && next_pair(p, b, hkv, j, i, g))) {
+            const int st = t & 1;
+            const int q0 = i * 128 + hh * 64;  // first query row of my 64 columns
+            const int qrow = b * p.Hq + hkv * p.G + g;
+            if (!warp_wait(&tl->qdo_full[st], (t >> 1) & 1, &tl->abort) ||
+                !warp_wait(&tl->s_full, t & 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
+            tc_fence_after();
+            const float *lse2 = &tl->lse2[st][hh * 64];
+            const float *delta = &tl->delta[st][hh * 64];
+            // last query column this key is visible to is unbounded unless causal:
+            // key <= q + shift  <=>  q >= key - shift
+            const int qmin = p.causal ? key - shift : INT_MIN;
+            const bool key_ok = key < p.Lk;
+            float pf[64];
+#pragma unroll
+            for (int c = 0; c < 2; c++) {
+                uint32_t sr[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(hh * 64 + c * 32), sr);
+                tc_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float v2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        const int cc = c * 32 + e + u;
+                        const bool vis = key_ok && (q0 + cc >= qmin);
+                        v2[u] = vis ? ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lse2[cc])) : 0.f;
+                        pf[cc] = v2[u];
+                    }
+                    pk[e >> 1] = pack_bf16x2(v2[0], v2[1]);
+                }
+                // P^T (bf16) over columns this thread has already read
+                tmem_st16(tmem + lane_off + (uint32_t)(hh * 64 + c * 16), pk);
+            }
+            if (!warp_wait(&tl->dp_full, t & 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
+            tc_fence_after();
+            // dS^T row r, my 64 queries -> box hh of sdS (128-byte swizzle, 8 chunks of 8 queries)
+            uint8_t *ds_row = sdS + hh * kBoxBytes;
+#pragma unroll
+            for (int c = 0; c < 2; c++) {
+                uint32_t dr[32];
+                tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * 64 + c * 32), dr);
+                tc_wait_ld();
+#pragma unroll
+                for (int ch = 0; ch < 4; ch++) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; u++) {
+                        const int cc = c * 32 + ch * 8 + 2 * u;
+                        const float d0 = p.scale * pf[cc] * (__uint_as_float(dr[ch * 8 + 2 * u]) - delta[cc]);
+                        const float d1 =
+                            p.scale * pf[cc + 1] * (__uint_as_float(dr[ch * 8 + 2 * u + 1]) - delta[cc + 1]);
+                        w[u] = pack_bf16x2(d0, d1);
+                    }
+                    *reinterpret_cast<uint4 *>(ds_row + swz128(r, c * 4 + ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            tc_wait_st();
+            fence_proxy_async();  // dS^T stores -> visible to the tensor core's reads
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->ds_ready);
+            // dQ^T(t): lane r is head dim r, columns my 64 queries
+            if (!warp_wait(&tl->dq_full, t & 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
+            tc_fence_after();
+            uint32_t qa[64];
+            tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * 64), qa);
+            tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * 64 + 32), qa + 32);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->dq_free);
+            float *acc = p.dq_acc + ((size_t)qrow * p.Lq_pad + q0) * 128 + r;
+            const int nvalid = min(64, p.Lq - q0);
+#pragma unroll
+            for (int c = 0; c < 64; c++)
+                if (c < nvalid) atomicAdd(acc + (size_t)c * 128, __uint_as_float(qa[c]));
+            t++;
+            advance(p, i, g);
+        }
+        n_steps = t;
+
+        // dK, dV of this block: lane r = key, my 64 head dims.  The TMEM loads are
+        // warp-collective (.sync.aligned): every lane issues them, and only the
+        // stores of keys past Lk (a partial last block) are left out.
+        if (__all_sync(0xffffffffu, !tl->abort) && warp_wait(&tl->acc_done, 0, &tl->abort)) {
+            tc_fence_after();
+            const bool store = key < p.Lk;
+            const size_t row_off = ((size_t)kvrow * p.Lk + (store ? key : 0)) * 128 + hh * 64;
+#pragma unroll
+            for (int m = 0; m < 2; m++) {
+                uint16_t *dst = (m ? p.dk : p.dv) + row_off;
+                const uint32_t col = (m ? 384u : 256u) + (uint32_t)(hh * 64);
+#pragma unroll
+                for (int c = 0; c < 2; c++) {
+                    uint32_t v[32];
+                    if (n_steps > 0) {  // warp-uniform
+                        tmem_ld32(tmem + lane_off + col + c * 32, v);
+                        tc_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; e++) v[e] = 0u;
+                    }
+                    if (store) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 o4;
+                            o4.x = pack_bf16x2(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1]));
+                            o4.y = pack_bf16x2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                            o4.z = pack_bf16x2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                            o4.w = pack_bf16x2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+                            *reinterpret_cast<uint4 *>(dst + c * 32 + e) = o4;
+                        }
+                    }
+                }
+            }
+        } else if (!tl->abort) {
+            set_timeout(tl, p.status);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// One warp per query row (padding rows included).
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 8 + warp;  // (b*Hq + hq) * Lq_pad + r
+    if (row >= (long long)p.B * p.Hq * p.Lq_pad) return;
+    const int r = (int)(row % p.Lq_pad);
+    const long long bh = row / p.Lq_pad;
+    float dsum = 0.f;
+    float l2 = CUDART_INF_F;
+    if (r < p.Lq) {
+        const size_t src = ((size_t)bh * p.Lq + r) * 128 + lane * 4;
+        const uint2 o2 = *reinterpret_cast<const uint2 *>(p.o + src);
+        const uint2 d2 = *reinterpret_cast<const uint2 *>(p.dout + src);
+        dsum = __uint_as_float(o2.x << 16) * __uint_as_float(d2.x << 16) +
+               __uint_as_float(o2.x & 0xFFFF0000u) * __uint_as_float(d2.x & 0xFFFF0000u) +
+               __uint_as_float(o2.y << 16) * __uint_as_float(d2.y << 16) +
+               __uint_as_float(o2.y & 0xFFFF0000u) * __uint_as_float(d2.y & 0xFFFF0000u);
+        const float lse = p.lse[(size_t)bh * p.Lq + r];
+        if (lse > -CUDART_INF_F) l2 = lse * 1.4426950408889634f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+    if (lane == 0) {
+        p.delta[row] = r < p.Lq ? dsum : 0.f;
+        p.lse2[row] = l2;
+    }
+    reinterpret_cast<float4 *>(p.dq_acc + row * 128)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dq = bf16(dQ accumulator), 4 elements per thread.
+__global__ void __launch_bounds__(256) bwd_finalize_kernel(const BwdParams p) {
+    const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;  // over B*Hq*Lq*32
+    if (idx >= (long long)p.B * p.Hq * p.Lq * 32) return;
+    const long long row = idx >> 5;  // (b*Hq + hq) * Lq + r
+    const int c4 = (int)(idx & 31);
+    const long long bh = row / p.Lq;
+    const int r = (int)(row % p.Lq);
+    const float4 a = reinterpret_cast<const float4 *>(p.dq_acc + ((size_t)bh * p.Lq_pad + r) * 128)[c4];
+    uint2 out;
+    out.x = pack_bf16x2(a.x, a.y);
+    out.y = pack_bf16x2(a.z, a.w);
+    reinterpret_cast<uint2 *>(p.dq + (size_t)row * 128)[c4] = out;
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
+                            const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st) {
+    const long long prep_rows = (long long)p.B * p.Hq * p.Lq_pad;
+    bwd_prep_kernel<<<(unsigned)((prep_rows + 7) / 8), 256, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.nb * p.Hkv, p.B);
+    bwd_kernel<<<grid, kThreads, kSmemBytes, st>>>(p, tq, tdo, tk, tv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long fin = (long long)p.B * p.Hq * p.Lq * 32;
+    bwd_finalize_kernel<<<(unsigned)((fin + 255) / 256), 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace blasst

@@ -382,9 +382,99 @@ blasst_status run_prefill(const void *q, const void *k, const void *v, void *o, 
     return BLASST_OK;
 }
 
+size_t backward_ws_parts(int B, int Hq, int Lq, size_t *acc_bytes, size_t *row_bytes) {
+    const size_t rows = (size_t)B * Hq * (size_t)(((long long)Lq + 127) / 128 * 128);
+    *acc_bytes = round_up(rows * 128 * sizeof(float), 256);
+    *row_bytes = round_up(rows * sizeof(float), 256);
+    return *acc_bytes + 2 * *row_bytes;
+}
+
+blasst_status run_backward(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                           const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Lq, int Lk,
+                           int d, float scale, int causal, const uint32_t *skip_mask, void *stream,
+                           const blasst_opts *opts_in) {
+    blasst_opts op = read_opts(opts_in);
+    Common c;
+    blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, 0.f, causal, op, &c);
+    if (st != BLASST_OK) return st;
+    if (!v || !o || !lse || !dout || !dq || !dk || !dv) return BLASST_ERR_INVALID;
+    if (!aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+        !aligned(dv, 16) || !aligned(lse, 4) || (skip_mask && !aligned(skip_mask, 4)))
+        return BLASST_ERR_INVALID;
+    if (op.seed_splits || op.mode) return BLASST_ERR_UNSUPPORTED;
+    if (op.block_n != 0 && op.block_n != kPrefillBlockN) return BLASST_ERR_UNSUPPORTED;
+    if (d != 128 || c.dv != 128 || c.krs != 128 || c.vrs != 128) return BLASST_ERR_UNSUPPORTED;
+    if (B > 65535) return BLASST_ERR_UNSUPPORTED;
+    const int nq = (Lq + kPrefillBlockM - 1) / kPrefillBlockM;
+    const int nb = (Lk + kPrefillBlockN - 1) / kPrefillBlockN;
+    if ((long long)nb * Hkv > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED;
+    size_t acc_bytes, row_bytes;
+    const size_t need = backward_ws_parts(B, Hq, Lq, &acc_bytes, &row_bytes);
+    void *ws = op.workspace;
+    if (ws && op.workspace_bytes < need) return BLASST_ERR_WORKSPACE;
+    cudaStream_t sm = reinterpret_cast<cudaStream_t>(stream);
+
+    CUtensorMap tq, tdo, tk, tv;
+    st = make_tmap(&tq, q, d, Lq, (long long)B * Hq, d, 64, kPrefillBlockM);
+    if (st != BLASST_OK) return st;
+    st = make_tmap(&tdo, dout, d, Lq, (long long)B * Hq, d, 64, kPrefillBlockM);
+    if (st != BLASST_OK) return st;
+    st = make_tmap(&tk, k, d, Lk, (long long)B * Hkv, d, 64, kPrefillBlockN);
+    if (st != BLASST_OK) return st;
+    st = make_tmap(&tv, v, d, Lk, (long long)B * Hkv, d, 64, kPrefillBlockN);
+    if (st != BLASST_OK) return st;
+    const bool own_ws = (ws == nullptr);
+    cudaError_t e;
+    if (own_ws) {
+        e = cudaMallocAsync(&ws, need, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+    }
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    BwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.o = static_cast<const uint16_t *>(o);
+    p.dout = static_cast<const uint16_t *>(dout);
+    p.lse = lse;
+    p.dq_acc = reinterpret_cast<float *>(w8);
+    p.lse2 = reinterpret_cast<float *>(w8 + acc_bytes);
+    p.delta = reinterpret_cast<float *>(w8 + acc_bytes + row_bytes);
+    p.dq = static_cast<uint16_t *>(dq);
+    p.dk = static_cast<uint16_t *>(dk);
+    p.dv = static_cast<uint16_t *>(dv);
+    p.skip_mask = skip_mask;
+    p.status = op.status_word;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.G = Hq / Hkv;
+    p.Lq_pad = nq * kPrefillBlockM; p.nq = nq; p.nb = nb; p.words = (nb + 31) / 32;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = (float)(scale * kLog2e);
+    p.scale = scale;
+    e = launch_backward(p, tq, tdo, tk, tv, sm);
+    blasst_status rs = BLASST_OK;
+    if (e != cudaSuccess) rs = cuda_fail(e, "backward kernels");
+    if (own_ws) {
+        cudaError_t e2 = cudaFreeAsync(ws, sm);
+        if (e2 != cudaSuccess && rs == BLASST_OK) rs = cuda_fail(e2, "cudaFreeAsync(workspace)");
+    }
+    return rs;
+}
+
 }  // namespace
 
 extern "C" {
+
+blasst_status blasst_prefill_backward(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                      const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,
+                                      int Lq, int Lk, int d, float scale, int causal, const uint32_t *skip_mask,
+                                      void *stream, const blasst_opts *opts) {
+    return run_backward(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Lq, Lk, d, scale, causal, skip_mask, stream,
+                        opts);
+}
+
+size_t blasst_backward_workspace_bytes(int B, int Hq, int Lq) {
+    if (B <= 0 || Hq <= 0 || Lq <= 0) return 0;
+    size_t a, r;
+    return backward_ws_parts(B, Hq, Lq, &a, &r);
+}
 
 blasst_status blasst_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                              int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,

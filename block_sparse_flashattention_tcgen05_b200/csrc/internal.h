@@ -59,6 +59,22 @@ struct PrefillParams {
     float thr_log2;
 };
 
+// One fixed-mask backward call (prefill tiling: 128-row query tiles, 128-key blocks, d = 128).
+struct BwdParams {
+    const uint16_t *o;              // [B, Hq, Lq, 128] bf16 forward output
+    const uint16_t *dout;           // [B, Hq, Lq, 128] bf16 upstream gradient
+    const float *lse;               // [B, Hq, Lq] forward lse (natural log)
+    float *lse2;                    // workspace [B*Hq, Lq_pad]: lse*log2(e), +inf on padding rows
+    float *delta;                   // workspace [B*Hq, Lq_pad]: rowsum(dO * O)
+    float *dq_acc;                  // workspace [B*Hq, Lq_pad, 128] fp32
+    uint16_t *dq;                   // [B, Hq, Lq, 128] bf16
+    uint16_t *dk, *dv;              // [B, Hkv, Lk, 128] bf16
+    const uint32_t *skip_mask;      // [B, Hq, nq, words] from the forward, or null (nothing skipped)
+    unsigned int *status;           // or null
+    int B, Hq, Hkv, Lq, Lk, G, Lq_pad, nq, nb, words, causal;
+    float scale_log2;               // scale * log2(e)
+    float scale;
+};
 // One MLA decode (or MLA-shaped calibration) call: a single latent KV head of
 // 576 columns, V = its first 512 columns.
 struct MlaParams {
@@ -76,6 +92,9 @@ struct MlaParams {
     float thr_log2;
 };
 
+// prep (delta, lse2, zeroed dQ accumulator), the main tcgen05 kernel, dq finalize
+cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_do,
+                            const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, cudaStream_t stream);
 // Records the text returned by blasst_last_error() for this thread.
 void set_last_error(const char *msg);
 

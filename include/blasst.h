@@ -164,6 +164,42 @@ BLASST_API blasst_status blasst_decode_paged(const void *q, const void *k_pages,
                                              unsigned long long *skip_count, void *stream, const blasst_opts *opts);
 
 /*
+ * Attention backward with the forward's skip mask held fixed (prefill tiling:
+ * query tiles of 128 rows of one query head, KV blocks of 128 keys, d = dv =
+ * 128).  The pages describe an optional sparsity-aware training in which the
+ * forward skips blocks and the skipped blocks receive no gradient (xllm-io
+ * paper review, section 3, "training procedure").  With the mask fixed the
+ * forward is plain masked softmax attention over the kept pairs, and this
+ * call returns its exact gradient up to rounding:
+ *   P = exp(scale*QK^T - lse) on kept, visible scores (0 elsewhere),
+ *   dV = P^T dO, dP = dO V^T, D = rowsum(dO * O), dS = P * (dP - D),
+ *   dQ = scale * dS K, dK = scale * dS^T Q  (dK, dV summed over the G query
+ *   heads of each KV head).
+ *
+ * q, k, v, o, lse  the forward's inputs and outputs (o, lse as blasst_prefill
+ *                  wrote them); dout [B, Hq, Lq, 128] bf16, the gradient of o.
+ * dq [B, Hq, Lq, 128], dk, dv [B, Hkv, Lk, 128]: bf16 outputs, fully written.
+ * skip_mask        the forward's mask (layout as above; blocks a tile never
+ *                  visits must read 0), or NULL: nothing skipped.
+ * causal           as in the forward.
+ * opts             workspace (>= blasst_backward_workspace_bytes() bytes,
+ *                  256-byte aligned; NULL -> stream-ordered cudaMallocAsync)
+ *                  and status_word; dv, strides and block_n must be defaults.
+ * Rounding: P and dS enter the tensor-core products as bf16, accumulation is
+ * fp32, dQ is accumulated across key blocks in an fp32 workspace by atomic
+ * adds (so the order of those additions, and the last bits of dq, can vary
+ * from run to run; dk and dv are deterministic).
+ */
+BLASST_API blasst_status blasst_prefill_backward(const void *q, const void *k, const void *v, const void *o,
+                                                 const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                                                 int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                                                 int causal, const uint32_t *skip_mask, void *stream,
+                                                 const blasst_opts *opts);
+/* Workspace of blasst_prefill_backward: an fp32 dQ accumulator and two fp32
+ * rows per query, padded to whole 128-row tiles.  0 for invalid sizes. */
+BLASST_API size_t blasst_backward_workspace_bytes(int B, int Hq, int Lq);
+
+/*
  * Calibration pass: the decision part of prefill (opts->mode = 0) or decode
  * (mode = 1) only -- QK^T, block row maxima, running max, gaps -- without
  * exp, P.V or V traffic.  v, o and lse may be NULL and are not touched.

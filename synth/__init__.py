@@ -51,9 +51,10 @@ __all__ = [
     "planted_prefill",
     "planted_decode",
     "planted_mla",
+    "upstream_grad",
 ]
 
-_TENSOR_ID = {"q": 1, "k": 2, "v": 3, "u": 4, "w": 5, "h": 6}
+_TENSOR_ID = {"q": 1, "k": 2, "v": 3, "u": 4, "w": 5, "h": 6, "do": 7}
 _CHUNK_ROWS = 1 << 14
 
 
@@ -295,3 +296,10 @@ def planted_mla(B, Hq, Lk, d_latent=512, d_rope=64, Lq=1, seed=0, reading="lit",
     meta = dict(kind="planted_mla", reading=reading, boost=boost, seed=seed, gamma=gamma,
                 d_latent=d_latent, d_rope=d_rope, heavy_fraction=float(HM.mean()))
     return AttnInputs(q, k, None, scale, meta)
+
+
+def upstream_grad(B, Hq, Lq, dv=128, seed=0) -> np.ndarray:
+    """Gradient of the attention output for the backward pass: iid N(0,1), bf16 bits."""
+    do = np.empty((B, Hq, Lq, dv), np.uint16)
+    _fill(do, seed, _TENSOR_ID["do"])
+    return do

@@ -111,6 +111,44 @@ def test_paged_decode_arguments_rejected_before_launch(bl):
     assert _paged(bl, opts=bl.Opts(k_row_stride=256)) == 2      # pages are dense rows
 
 
+def _bwd(bl, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, do=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, Hq=4, Hkv=2, Lq=256,
+             Lk=256, d=128, scale=0.088, causal=1, mask=None)
+    a.update(over)
+    return bl.lib().blasst_prefill_backward(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"],
+                                            a["dv"], a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"], a["d"],
+                                            a["scale"], a["causal"], a["mask"], None,
+                                            ctypes.byref(a.get("opts") or bl.Opts()))
+
+
+def test_backward_arguments_rejected_before_launch(bl):
+    for name in ("q", "k", "v", "o", "lse", "do", "dq", "dk", "dv"):
+        assert _bwd(bl, **{name: None}) == 1, name
+    for name in ("q", "k", "v", "o", "do", "dq", "dk", "dv"):
+        assert _bwd(bl, **{name: FAKE + 8}) == 1, name
+    assert _bwd(bl, lse=FAKE + 2) == 1
+    assert _bwd(bl, mask=FAKE + 2) == 1
+    assert _bwd(bl, Hq=3) == 1                      # Hq not a multiple of Hkv
+    assert _bwd(bl, Lq=300, Lk=256) == 1            # causal needs Lq <= Lk
+    assert _bwd(bl, scale=-1.0) == 1
+    assert _bwd(bl, d=64) == 2
+    assert _bwd(bl, opts=bl.Opts(dv=64)) == 2
+    assert _bwd(bl, opts=bl.Opts(k_row_stride=256)) == 2
+    assert _bwd(bl, opts=bl.Opts(block_n=64)) == 2
+    assert _bwd(bl, opts=bl.Opts(seed_splits=1)) == 2
+    assert _bwd(bl, opts=bl.Opts(workspace=FAKE, workspace_bytes=64)) == 3
+    assert _bwd(bl, opts=bl.Opts(workspace=FAKE + 16, workspace_bytes=1 << 30)) == 1
+
+
+def test_backward_workspace_bytes(bl):
+    f = bl.lib().blasst_backward_workspace_bytes
+    # 2 x 32 rows padded to 2 tiles: fp32 accumulator of 128 columns + two fp32 rows, 256-byte rounded
+    rows = 2 * 32 * 256
+    assert f(2, 32, 200) == rows * 128 * 4 + 2 * rows * 4
+    assert f(1, 1, 1) == 128 * 128 * 4 + 2 * 512
+    assert f(0, 1, 1) == 0 and f(1, 1, 0) == 0
+
+
 def test_calibrate_requires_gaps_and_valid_mode(bl):
     assert _call(bl, "blasst_calibrate") == 1                 # no gaps_out
     assert _call(bl, "blasst_calibrate", opts=bl.Opts(mode=7, gaps_out=FAKE)) == 1

@@ -5,8 +5,8 @@
 // skipped blocks receive no gradient in the backward pass).
 //
 // Three launches:
-//   prep      per query row: delta = rowsum(dO * O) (fp32), lse2 = lse*log2(e)
-//             (+inf on padding rows and rows that saw no key, so their P is 0),
+//   prep      per query row: -scale * rowsum(dO * O) and -lse*log2(e) (fp32;
+//             -inf on padding rows and rows that saw no key, so their P is 0),
 //             and the row of the fp32 dQ accumulator set to zero;
 //   main      one CTA per (KV block j of 128 keys, KV head, sequence) walks the
 //             kept (query tile i, query head) pairs of its KV head in order
@@ -18,21 +18,23 @@
 // Main kernel, per pair (S^T etc. are key-major: TMEM lane = key of block j):
 //   S^T  = K_j Q_i^T                        tcgen05, A = K (K-major), B = Q (K-major)
 //   dP^T = V_j dO_i^T                       tcgen05, A = V, B = dO (both K-major)
-//   P^T  = 2^(S^T * scale*log2e - lse2)     masked (key >= Lk, causal) to 0
-//   dS^T = scale * P^T (dP^T - delta)       bf16 into shared memory
+//   P^T  = 2^(S^T * scale*log2e - lse*log2e)  masked (key >= Lk, causal) to 0
+//   dS^T = P^T (scale*dP^T - scale*D)       bf16 into shared memory
 //   dQ^T = K_j^T dS^T                       A = K (MN-major), B = dS^T (MN-major)
 //   dV  += P^T dO_i                         A = P^T from TMEM (bf16), B = dO (MN-major)
 //   dK  += dS^T Q_i                         A = dS^T (K-major), B = Q (MN-major)
 //
-// Warp roles (320 threads):
-//   warps 0-7  compute: warp w owns TMEM lanes 32*(w%4).. (keys for S^T/dP^T,
-//              head dims for dQ^T) and query half w/4 (64 columns);
-//   warp 8     TMA producer: K_j, V_j once; Q_i, dO_i, lse2_i, delta_i per pair
-//              into a 2-stage ring;
-//   warp 9     allocates TMEM and issues every tcgen05.mma from one thread.
+// Warp roles:
+//   compute    4 * kColGroups warps: warp w owns TMEM lanes 32*(w%4).. (keys
+//              for S^T/dP^T, head dims for dQ^T) and column group w/4 (128 /
+//              kColGroups columns);
+//   producer   TMA: K_j, V_j once; Q_i, dO_i and the two per-row vectors per
+//              pair into a 2-stage ring;
+//   MMA        allocates TMEM and issues every tcgen05.mma from one thread.
 //
-// TMEM (512 columns): S^T [0,128) -> P^T (bf16; queries 0-63 in [0,32),
-// 64-127 in [64,96)); dP^T [128,256) -> dQ^T; dV [256,384); dK [384,512).
+// TMEM (512 columns): S^T [0,128) -> P^T (bf16; each column group's P^T packed
+// into the first half of its own S^T columns); dP^T [128,256) -> dQ^T;
+// dV [256,384); dK [384,512).
 //
 // MMA issue order per pair t: dP(t) [after the dQ^T(t-1) columns are read],
 // then, once dS^T(t) is ready: dQ^T(t), dV(t), S(t+1), dK(t).  The compute
@@ -50,18 +52,27 @@
 namespace blasst {
 namespace {
 
-constexpr int kComputeWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+#ifndef BLASST_BWD_COL_GROUPS
+#define BLASST_BWD_COL_GROUPS 4
+#endif
+// The 128 columns of a pair are split into kColGroups groups; a compute warp owns
+// one TMEM lane quadrant and one group, so there are 4 * kColGroups compute warps.
+constexpr int kColGroups = BLASST_BWD_COL_GROUPS;
+constexpr int kCW = 128 / kColGroups;  // columns per compute warp (64 or 32)
+constexpr int kChunks = kCW / 32;      // 32-column TMEM loads per operand
+constexpr int kComputeWarps = 4 * kColGroups;
+constexpr int kProducerWarp = kComputeWarps;
+constexpr int kMmaWarp = kComputeWarps + 1;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
+static_assert(kColGroups == 2 || kColGroups == 4, "64 or 32 columns per compute warp");
 constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
 constexpr int kBoxBytes = kTileBytes / 2;  // 128 rows x 64 bf16 (one 128-byte swizzle box)
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusSmemAlign = 4;
 
 struct BwdTail {
-    float lse2[2][128];   // per stage: lse * log2(e) of the pair's 128 query rows
-    float delta[2][128];  // per stage: rowsum(dO * O)
+    float nl2[2][128];  // per stage: -lse * log2(e) of the pair's 128 query rows
+    float nsd[2][128];  // per stage: -scale * rowsum(dO * O)
     uint64_t kv_full;
     uint64_t qdo_full[2], qdo_empty[2];
     uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
@@ -190,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(q_dst + kBoxBytes, &tmap_q, &tl->qdo_full[st], 64, i * 128, qrow);
                 tma_load_3d(do_dst, &tmap_do, &tl->qdo_full[st], 0, i * 128, qrow);
                 tma_load_3d(do_dst + kBoxBytes, &tmap_do, &tl->qdo_full[st], 64, i * 128, qrow);
-                bulk_load(&tl->lse2[st][0], p.lse2 + rbase, 512, &tl->qdo_full[st]);
-                bulk_load(&tl->delta[st][0], p.delta + rbase, 512, &tl->qdo_full[st]);
+                bulk_load(&tl->nl2[st][0], p.neg_lse2 + rbase, 512, &tl->qdo_full[st]);
+                bulk_load(&tl->nsd[st][0], p.neg_sdelta + rbase, 512, &tl->qdo_full[st]);
                 t++;
                 advance(p, i, g);
             }
@@ -251,6 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < 8; kk++)
                     umma_ss2(tmem + 128, v_km + koff(kk), do_km + st * kStage16 + koff(kk), dhi, idesc_kk, kk > 0);
                 umma_commit(&tl->dp_full);
+                // the next pair (a mask lookup in global memory) while dS^T(t) is formed
+                int ni = i, ng = g;
+                advance(p, ni, ng);
+                const bool more = next_pair(p, b, hkv, j, ni, ng);
+                const int nst = (t + 1) & 1;
                 if (!mbar_wait(&tl->ds_ready, t & 1, &tl->abort)) {
                     set_timeout(tl, p.status);
                     break;
@@ -261,18 +277,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < 8; kk++)
                     umma_ss2(tmem + 128, k_mn + kk * (2048 >> 4), ds_mn + kk * (2048 >> 4), dhi, idesc_mnmn, kk > 0);
                 umma_commit(&tl->dq_full);
-                // dV += P^T dO (K = 128 queries; P^T halves at TMEM columns 0 and 64)
+                // dV += P^T dO (K = 128 queries; P^T of each column group in its own S^T columns)
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++)
-                    umma_ts2(tmem + 256, tmem + (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8),
+                    umma_ts2(tmem + 256, tmem + (uint32_t)((kk * 16 / kCW) * kCW + (kk * 16 % kCW) / 2),
                              do_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn, (t > 0 || kk > 0) ? 1u : 0u);
-                // next pair's S^T, so that its softmax overlaps dK(t) and dP(t+1)
-                int ni = i, ng = g;
-                advance(p, ni, ng);
-                const bool more = next_pair(p, b, hkv, j, ni, ng);
+                auto issue_dk = [&]() {  // dK += dS^T Q (K = 128 queries)
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++)
+                        umma_ss2(tmem + 384, ds_km + koff(kk), q_mn + st * kStage16 + kk * (2048 >> 4), dhi,
+                                 idesc_kmn, (t > 0 || kk > 0) ? 1u : 0u);
+                };
+                // The next pair's S^T goes ahead of dK(t) when its Q tile has landed, so that its
+                // exponentials overlap dK(t) and dP(t+1); otherwise dK(t) keeps the pipe busy first.
+                bool dk_done = false;
                 if (more) {
-                    const int nst = (t + 1) & 1;
-                    if (!mbar_wait(&tl->qdo_full[nst], ((t + 1) >> 1) & 1, &tl->abort)) {
+                    const uint32_t npar = ((t + 1) >> 1) & 1;
+                    if (!mbar_test_wait(&tl->qdo_full[nst], npar)) {
+                        issue_dk();
+                        dk_done = true;
+                    }
+                    if (!mbar_wait(&tl->qdo_full[nst], npar, &tl->abort)) {
                         set_timeout(tl, p.status);
                         break;
                     }
@@ -280,11 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issue_s(nst);
                     umma_commit(&tl->s_full);
                 }
-                // dK += dS^T Q (K = 128 queries)
-#pragma unroll
-                for (int kk = 0; kk < 8; kk++)
-                    umma_ss2(tmem + 384, ds_km + koff(kk), q_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn,
-                             (t > 0 || kk > 0) ? 1u : 0u);
+                if (!dk_done) issue_dk();
                 umma_commit(&tl->qdo_empty[st]);
                 t++;
                 i = ni;
@@ -298,15 +319,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ compute warps
         const int wq = warp & 3;   // TMEM lane quadrant
-        const int hh = warp >> 2;  // query half: columns 64*hh .. 64*hh+63
-        const int r = wq * 32 + lane;  // key row within the block (S^T, dP^T), head dim (dQ^T)
+        const int hh = warp >> 2;  // column group: columns kCW*hh .. kCW*hh + kCW - 1
+        const int r = wq * 32 + lane;  // TMEM lane: key row of the block (S^T, dP^T), head dim (dQ^T)
         const int key = j * 128 + r;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const int shift = p.Lk - p.Lq;
         int i = first_tile(p, j), g = 0, t = 0;
         while (__all_sync(0xffffffffu, !tl->abort && next_pair(p, b, hkv, j, i, g))) {
             const int st = t & 1;
-            const int q0 = i * 128 + hh * 64;  // first query row of my 64 columns
+            const int q0 = i * 128 + hh * kCW;  // first query row of my columns
             const int qrow = b * p.Hq + hkv * p.G + g;
             if (!warp_wait(&tl->qdo_full[st], (t >> 1) & 1, &tl->abort) ||
                 !warp_wait(&tl->s_full, t & 1, &tl->abort)) {
@@ -314,58 +335,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const float *lse2 = &tl->lse2[st][hh * 64];
-            const float *delta = &tl->delta[st][hh * 64];
-            // last query column this key is visible to is unbounded unless causal:
-            // key <= q + shift  <=>  q >= key - shift
-            const int qmin = p.causal ? key - shift : INT_MIN;
+            const float *nl2 = &tl->nl2[st][hh * kCW];
+            const float *nsd = &tl->nsd[st][hh * kCW];
+            // Masking is needed only where some key of the block is past Lk or, causal,
+            // past the first query of my columns (key <= q + shift); warp-uniform.
+            const bool masked = (j * 128 + 128 > p.Lk) || (p.causal && j * 128 + 127 > q0 + shift);
+            const int qmin = p.causal ? key - shift : INT_MIN;  // visible iff q >= qmin
             const bool key_ok = key < p.Lk;
-            float pf[64];
+            const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+            uint64_t pf[kCW / 2];  // P of my columns, as packed pairs
 #pragma unroll
-            for (int c = 0; c < 2; c++) {
+            for (int c = 0; c < kChunks; c++) {
                 uint32_t sr[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(hh * 64 + c * 32), sr);
+                tmem_ld32(tmem + lane_off + (uint32_t)(hh * kCW + c * 32), sr);
                 tc_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    float v2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; u++) {
-                        const int cc = c * 32 + e + u;
-                        const bool vis = key_ok && (q0 + cc >= qmin);
-                        v2[u] = vis ? ex2(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lse2[cc])) : 0.f;
-                        pf[cc] = v2[u];
+                    const int cc = c * 32 + e;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2,
+                                     *reinterpret_cast<const uint64_t *>(nl2 + cc)),
+                              x0, x1);
+                    if (masked) {
+                        if (!(key_ok && q0 + cc >= qmin)) x0 = -CUDART_INF_F;
+                        if (!(key_ok && q0 + cc + 1 >= qmin)) x1 = -CUDART_INF_F;
                     }
-                    pk[e >> 1] = pack_bf16x2(v2[0], v2[1]);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    pf[cc >> 1] = f2_pack(p0, p1);
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
                 }
                 // P^T (bf16) over columns this thread has already read
-                tmem_st16(tmem + lane_off + (uint32_t)(hh * 64 + c * 16), pk);
+                tmem_st16(tmem + lane_off + (uint32_t)(hh * kCW + c * 16), pk);
             }
             if (!warp_wait(&tl->dp_full, t & 1, &tl->abort)) {
                 set_timeout(tl, p.status);
                 break;
             }
             tc_fence_after();
-            // dS^T row r, my 64 queries -> box hh of sdS (128-byte swizzle, 8 chunks of 8 queries)
-            uint8_t *ds_row = sdS + hh * kBoxBytes;
+            // dS^T row r, my queries -> their 64-query box of sdS (128-byte swizzle, chunks of 8 queries)
+            uint8_t *ds_row = sdS + (hh * kCW / 64) * kBoxBytes;
+            const int chunk0 = (hh * kCW % 64) / 8;
+            const uint64_t sc2 = f2_pack(p.scale, p.scale);
 #pragma unroll
-            for (int c = 0; c < 2; c++) {
+            for (int c = 0; c < kChunks; c++) {
                 uint32_t dr[32];
-                tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * 64 + c * 32), dr);
+                tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * kCW + c * 32), dr);
                 tc_wait_ld();
 #pragma unroll
                 for (int ch = 0; ch < 4; ch++) {
                     uint32_t w[4];
 #pragma unroll
                     for (int u = 0; u < 4; u++) {
-                        const int cc = c * 32 + ch * 8 + 2 * u;
-                        const float d0 = p.scale * pf[cc] * (__uint_as_float(dr[ch * 8 + 2 * u]) - delta[cc]);
-                        const float d1 =
-                            p.scale * pf[cc + 1] * (__uint_as_float(dr[ch * 8 + 2 * u + 1]) - delta[cc + 1]);
+                        const int e = ch * 8 + 2 * u;
+                        const int cc = c * 32 + e;
+                        // dS = P * (scale*dP - scale*D)
+                        const uint64_t t2 = f2_fma(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), sc2,
+                                                   *reinterpret_cast<const uint64_t *>(nsd + cc));
+                        float d0, d1;
+                        f2_unpack(f2_mul(t2, pf[cc >> 1]), d0, d1);
                         w[u] = pack_bf16x2(d0, d1);
                     }
-                    *reinterpret_cast<uint4 *>(ds_row + swz128(r, c * 4 + ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(ds_row + swz128(r, chunk0 + c * 4 + ch)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             tc_wait_st();
@@ -379,17 +411,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t qa[64];
-            tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * 64), qa);
-            tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * 64 + 32), qa + 32);
+            uint32_t qa[kCW];
+#pragma unroll
+            for (int c = 0; c < kChunks; c++) tmem_ld32(tmem + 128 + lane_off + (uint32_t)(hh * kCW + c * 32), qa + c * 32);
             tc_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tl->dq_free);
+            // a warp adds 128 contiguous bytes (32 head dims of one query row) per instruction
             float *acc = p.dq_acc + ((size_t)qrow * p.Lq_pad + q0) * 128 + r;
-            const int nvalid = min(64, p.Lq - q0);
+            const int nvalid = min(kCW, p.Lq - q0);
 #pragma unroll
-            for (int c = 0; c < 64; c++)
+            for (int c = 0; c < kCW; c++)
                 if (c < nvalid) atomicAdd(acc + (size_t)c * 128, __uint_as_float(qa[c]));
             t++;
             advance(p, i, g);
@@ -402,13 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__all_sync(0xffffffffu, !tl->abort) && warp_wait(&tl->acc_done, 0, &tl->abort)) {
             tc_fence_after();
             const bool store = key < p.Lk;
-            const size_t row_off = ((size_t)kvrow * p.Lk + (store ? key : 0)) * 128 + hh * 64;
+            const size_t row_off = ((size_t)kvrow * p.Lk + (store ? key : 0)) * 128 + hh * kCW;
 #pragma unroll
             for (int m = 0; m < 2; m++) {
                 uint16_t *dst = (m ? p.dk : p.dv) + row_off;
-                const uint32_t col = (m ? 384u : 256u) + (uint32_t)(hh * 64);
+                const uint32_t col = (m ? 384u : 256u) + (uint32_t)(hh * kCW);
 #pragma unroll
-                for (int c = 0; c < 2; c++) {
+                for (int c = 0; c < kChunks; c++) {
                     uint32_t v[32];
                     if (n_steps > 0) {  // warp-uniform
                         tmem_ld32(tmem + lane_off + col + c * 32, v);
@@ -449,7 +482,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
     const int r = (int)(row % p.Lq_pad);
     const long long bh = row / p.Lq_pad;
     float dsum = 0.f;
-    float l2 = CUDART_INF_F;
+    float nl2 = -CUDART_INF_F;
     if (r < p.Lq) {
         const size_t src = ((size_t)bh * p.Lq + r) * 128 + lane * 4;
         const uint2 o2 = *reinterpret_cast<const uint2 *>(p.o + src);
@@ -459,13 +492,13 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
                __uint_as_float(o2.y << 16) * __uint_as_float(d2.y << 16) +
                __uint_as_float(o2.y & 0xFFFF0000u) * __uint_as_float(d2.y & 0xFFFF0000u);
         const float lse = p.lse[(size_t)bh * p.Lq + r];
-        if (lse > -CUDART_INF_F) l2 = lse * 1.4426950408889634f;
+        if (lse > -CUDART_INF_F) nl2 = -lse * 1.4426950408889634f;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
     if (lane == 0) {
-        p.delta[row] = r < p.Lq ? dsum : 0.f;
-        p.lse2[row] = l2;
+        p.neg_sdelta[row] = r < p.Lq ? -p.scale * dsum : 0.f;
+        p.neg_lse2[row] = nl2;
     }
     reinterpret_cast<float4 *>(p.dq_acc + row * 128)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
 }

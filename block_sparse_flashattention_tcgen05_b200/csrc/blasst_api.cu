@@ -436,8 +436,8 @@ blasst_status run_backward(const void *q, const void *k, const void *v, const vo
     p.dout = static_cast<const uint16_t *>(dout);
     p.lse = lse;
     p.dq_acc = reinterpret_cast<float *>(w8);
-    p.lse2 = reinterpret_cast<float *>(w8 + acc_bytes);
-    p.delta = reinterpret_cast<float *>(w8 + acc_bytes + row_bytes);
+    p.neg_lse2 = reinterpret_cast<float *>(w8 + acc_bytes);
+    p.neg_sdelta = reinterpret_cast<float *>(w8 + acc_bytes + row_bytes);
     p.dq = static_cast<uint16_t *>(dq);
     p.dk = static_cast<uint16_t *>(dk);
     p.dv = static_cast<uint16_t *>(dv);

@@ -64,8 +64,8 @@ struct BwdParams {
     const uint16_t *o;              // [B, Hq, Lq, 128] bf16 forward output
     const uint16_t *dout;           // [B, Hq, Lq, 128] bf16 upstream gradient
     const float *lse;               // [B, Hq, Lq] forward lse (natural log)
-    float *lse2;                    // workspace [B*Hq, Lq_pad]: lse*log2(e), +inf on padding rows
-    float *delta;                   // workspace [B*Hq, Lq_pad]: rowsum(dO * O)
+    float *neg_lse2;                // workspace [B*Hq, Lq_pad]: -lse*log2(e), -inf on padding rows
+    float *neg_sdelta;              // workspace [B*Hq, Lq_pad]: -scale * rowsum(dO * O)
     float *dq_acc;                  // workspace [B*Hq, Lq_pad, 128] fp32
     uint16_t *dq;                   // [B, Hq, Lq, 128] bf16
     uint16_t *dk, *dv;              // [B, Hkv, Lk, 128] bf16

@@ -283,8 +283,32 @@ class Backward(Prefill):
         return 5 * FLOP_PER_PAIR * (self.visited - skipped)
 
     def host_bytes(self):
-        return (self.inp.q.nbytes * 3 + self.inp.k.nbytes + self.inp.v.nbytes + self.lse.numel() * 4,
-                self.inp.q.nbytes + self.inp.k.nbytes * 2)
+        return (self.inp.q.nbytes * 3 + self.inp.k.nbytes + self.inp.v.nbytes + self.lse.numel() * 4 +
+                self.mask.numel() * 4, self.inp.q.nbytes + self.inp.k.nbytes * 2)
+
+    def e2e_call(self, lam, hq, hk, hv, ho, hl):
+        """Every input from pinned host memory (q, k, v and the forward's o, lse, mask, plus dout),
+        the backward through the public API, dq, dk, dv back to the host."""
+        import torch
+
+        if getattr(self, "_host", None) is None or self._host[0] != lam:
+            self.count = torch.zeros(1, dtype=torch.int64, device=self.device)
+            self.forward(lam)
+            pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+            self._host = (lam, pin(self.o), pin(self.lse), pin(self.mask), pin(self.dout),
+                          torch.empty(self.q.shape, dtype=torch.bfloat16).pin_memory(),
+                          torch.empty(self.k.shape, dtype=torch.bfloat16).pin_memory(),
+                          torch.empty(self.v.shape, dtype=torch.bfloat16).pin_memory())
+        _, h_o, h_lse, h_mask, h_do, h_dq, h_dk, h_dv = self._host
+        for dst, src in ((self.q, hq), (self.k, hk), (self.v, hv), (self.o, h_o), (self.lse, h_lse),
+                         (self.mask, h_mask), (self.dout, h_do)):
+            dst.copy_(src, non_blocking=True)
+        self.bl.prefill_backward(self.q, self.k, self.v, self.o, self.lse, self.dout, scale=self.inp.scale,
+                                 causal=True, skip_mask=self.mask, dq=self.dq, dk=self.dk, dv=self.dv,
+                                 workspace=self.ws)
+        h_dq.copy_(self.dq, non_blocking=True)
+        h_dk.copy_(self.dk, non_blocking=True)
+        h_dv.copy_(self.dv, non_blocking=True)
 
 
 class Decode:

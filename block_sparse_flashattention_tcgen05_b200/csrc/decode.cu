@@ -91,7 +91,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     DecodeSmemTail *tl = reinterpret_cast<DecodeSmemTail *>(vring + (CALIB ? 0 : NV * kStageBytes));
     volatile uint8_t *dec = reinterpret_cast<volatile uint8_t *>(tl + 1);
 
-    const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    // CTA order: every (sequence, KV head)'s first split, then its last split, then the middle ones.
+    // The first and last chunks hold the sink and the most recent keys, where kept blocks gather,
+    // so the CTAs with the most V traffic start early and the tail of the grid is made of the rest.
+    int split, hkv, b;
+    {
+        const int groups = p.Hkv * p.B;
+        const int L = blockIdx.x;
+        int grp;
+        if (L < groups) {
+            split = 0;
+            grp = L;
+        } else if (p.num_splits > 1 && L < 2 * groups) {
+            split = p.num_splits - 1;
+            grp = L - groups;
+        } else {
+            const int m = L - min(2, p.num_splits) * groups;
+            split = 1 + m / groups;
+            grp = m % groups;
+        }
+        hkv = grp % p.Hkv;
+        b = grp / p.Hkv;
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // keys of this sequence: all Lk, or (paged) its own length, split the same way
     int Lk = p.Lk, nbs = p.nb, per_split = p.per_split;
@@ -585,8 +606,7 @@ cudaError_t launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const 
     auto kern = decode_split_kernel<NT, NK, NV, CALIB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.num_splits, p.Hkv, p.B);
-    kern<<<grid, kThreads, smem, st>>>(p, tk, tv);
+    kern<<<p.num_splits * p.Hkv * p.B, kThreads, smem, st>>>(p, tk, tv);
     return cudaGetLastError();
 }
 

@@ -13,7 +13,7 @@ import os
 __all__ = [
     "BlasstError", "lib", "prefill", "decode", "decode_noalloc", "calibrate", "calibrate_fit", "calibrate_threshold",
     "visited_pairs", "decode_workspace_bytes", "mask_words", "Opts", "STATUS", "prefill_backward",
-    "backward_workspace_bytes",
+    "backward_workspace_bytes", "decode_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -81,6 +81,10 @@ def lib() -> ctypes.CDLL:
         L.blasst_decode_paged.argtypes = ([ctypes.c_void_p] * 7 + [ctypes.c_int] * 7 +
                                           [ctypes.c_float, ctypes.c_float, ctypes.c_int] + [ctypes.c_void_p] * 3 +
                                           [ctypes.POINTER(Opts)])
+        L.blasst_decode_fp8.restype = ctypes.c_int
+        L.blasst_decode_fp8.argtypes = ([ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 +
+                                        [ctypes.c_float] * 4 + [ctypes.c_int] + [ctypes.c_void_p] * 3 +
+                                        [ctypes.POINTER(Opts)])
         L.blasst_prefill_backward.restype = ctypes.c_int
         L.blasst_prefill_backward.argtypes = ([ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 +
                                               [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
@@ -249,6 +253,39 @@ def decode(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o
                  want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hkv,
                  n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=dv)
     return o, lse, m, c
+
+
+def decode_fp8(q, k8, v8, *, scale, k_scale, v_scale, lam=0.0, causal=False, num_splits=None, o=None, lse=None,
+               skip_mask=True, skip_count=True, workspace=None, status_word=None, stream=None, seed_splits=False):
+    """Split-KV decode over an FP8 (e4m3) cache: K = k_scale * k8, V = v_scale * v8.
+
+    q [B,Hq,Lq,128] bf16; k8, v8 [B,Hkv,Lk,128] uint8 (or float8_e4m3fn) on CUDA; (Hq/Hkv)*Lq <= 16.
+    Returns (o, lse, skip_mask [B*Hkv, W] int32 or None, skip_count [1] int64 or None).
+    """
+    import torch
+
+    _dev_tensor(q, "q"), _dev_tensor(k8, "k8"), _dev_tensor(v8, "v8")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k8.shape
+    if o is None:
+        o = torch.empty((B, Hq, Lq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    opts = Opts(num_splits=num_splits or 0, status_word=None if status_word is None else status_word.data_ptr(),
+                seed_splits=int(bool(seed_splits)))
+    if workspace is not None:
+        opts.workspace = workspace.data_ptr()
+        opts.workspace_bytes = workspace.numel() * workspace.element_size()
+    nb = (Lk + 63) // 64
+    mask = torch.empty((B * Hkv, mask_words(nb)), dtype=torch.int32, device=q.device) if skip_mask is True else (
+        skip_mask if isinstance(skip_mask, torch.Tensor) else None)
+    count = torch.empty(1, dtype=torch.int64, device=q.device) if skip_count is True else (
+        skip_count if isinstance(skip_count, torch.Tensor) else None)
+    rc = lib().blasst_decode_fp8(_ptr(q), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, d,
+                                 float(scale), float(k_scale), float(v_scale), float(lam), int(bool(causal)),
+                                 _ptr(mask), _ptr(count), _stream(stream), ctypes.byref(opts))
+    _check(rc, "blasst_decode_fp8")
+    return o, lse, mask, count
 
 
 def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=None, skip_mask=True,

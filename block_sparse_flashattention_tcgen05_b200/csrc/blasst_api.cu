@@ -69,6 +69,27 @@ blasst_status make_tmap(CUtensorMap *m, const void *base, long long cols, long l
     return BLASST_OK;
 }
 
+// 3-D view of an e4m3 (byte) cache [outer, rows, 128]: one 128-byte-swizzled box of 128 x box_rows.
+blasst_status make_tmap_u8(CUtensorMap *m, const void *base, long long rows, long long outer, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return BLASST_ERR_CUDA;
+    }
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)outer};
+    cuuint64_t strides[2] = {128, (cuuint64_t)rows * 128};
+    cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return BLASST_ERR_CUDA;
+    }
+    return BLASST_OK;
+}
+
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Copy of the caller's options with fields past struct_size zeroed.
@@ -198,10 +219,15 @@ struct PagedCache {
     int max_pages, num_pages;
 };
 
+// FP8 (e4m3) K/V cache: K = k_scale * e4m3, V = v_scale * e4m3.
+struct Fp8Cache {
+    float k_scale, v_scale;
+};
+
 blasst_status run_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                          int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
                          unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib,
-                         const PagedCache *pg = nullptr) {
+                         const PagedCache *pg = nullptr, const Fp8Cache *f8 = nullptr) {
     blasst_opts op = read_opts(opts_in);
     Common c;
     blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, op, &c);
@@ -215,6 +241,12 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     if (op.block_n != 0 && op.block_n != kDecodeBlockN) return BLASST_ERR_UNSUPPORTED;
     if (op.seed_splits && d != 128) return BLASST_ERR_UNSUPPORTED;  // split seeding: GQA/MQA decode only
     if (pg && (d != 128 || c.dv != 128 || c.krs != d || c.vrs != c.dv)) return BLASST_ERR_UNSUPPORTED;
+    if (f8) {
+        if (!(std::isfinite(f8->k_scale) && f8->k_scale > 0.f && std::isfinite(f8->v_scale) && f8->v_scale > 0.f))
+            return BLASST_ERR_INVALID;
+        if (calib || pg || d != 128 || c.dv != 128 || c.krs != d || c.vrs != c.dv) return BLASST_ERR_UNSUPPORTED;
+        if ((long long)(Hq / Hkv) * Lq > 16) return BLASST_ERR_UNSUPPORTED;  // tiles of up to 16 rows
+    }
     if (d == 576) return run_mla(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count,
                                  stream, op, c, calib);
     if (d != 128 || c.dv != 128) return BLASST_ERR_UNSUPPORTED;
@@ -246,13 +278,19 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     const long long planes = pg ? (long long)pg->num_pages * Hkv : (long long)B * Hkv;
     const long long plane_rows = pg ? kDecodeBlockN : Lk;
     CUtensorMap tk, tv;
-    st = make_tmap(&tk, k, d, plane_rows, planes, c.krs, 64, 64);
-    if (st != BLASST_OK) return st;
-    if (!calib) {
-        st = make_tmap(&tv, v, c.dv, plane_rows, planes, c.vrs, 64, 64);
+    if (f8) {  // e4m3 rows of 128 bytes
+        st = make_tmap_u8(&tk, k, plane_rows, planes, 64);
+        if (st == BLASST_OK) st = make_tmap_u8(&tv, v, plane_rows, planes, 64);
         if (st != BLASST_OK) return st;
     } else {
-        tv = tk;
+        st = make_tmap(&tk, k, d, plane_rows, planes, c.krs, 64, 64);
+        if (st != BLASST_OK) return st;
+        if (!calib) {
+            st = make_tmap(&tv, v, c.dv, plane_rows, planes, c.vrs, 64, 64);
+            if (st != BLASST_OK) return st;
+        } else {
+            tv = tk;
+        }
     }
     CUtensorMap tq;  // wide tiles: q as [B][Hq*Lq][128], 128-row boxes
     if (wide) {
@@ -281,7 +319,6 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
     p.q = static_cast<const uint16_t *>(q);
-    p.q = static_cast<const uint16_t *>(q);
     p.part_o = calib ? nullptr : static_cast<float *>(ws);
     p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));
     p.skip_mask = skip_mask;
@@ -291,15 +328,18 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.G = G; p.R = (int)R;
     p.nb = nb; p.num_splits = S; p.per_split = per_split; p.words = words;
     p.causal = causal ? 1 : 0;
-    p.scale_log2 = (float)(scale * kLog2e);
+    p.scale_log2 = (float)(scale * kLog2e * (f8 ? f8->k_scale : 1.f));
     p.thr_log2 = log2_threshold(lambda);
     p.seed = op.seed_splits ? 1 : 0;
+    p.v_scale = f8 ? f8->v_scale : 1.f;
     if (pg) {
         p.block_table = pg->block_table;
         p.seq_lens = pg->seq_lens;
         p.num_pages = pg->num_pages;
     }
-    if (wide) {
+    if (f8) {
+        e = launch_decode_fp8(p, tk, tv, R <= 8 ? 1 : 2, sm);
+    } else if (wide) {
         e = launch_decode_wide(p, tq, tk, tv, calib, sm);
     } else {
         e = launch_decode(p, tk, tv, calib, R <= 8 ? 1 : 2, sm);
@@ -488,6 +528,16 @@ blasst_status blasst_decode(const void *q, const void *k, const void *v, void *o
                             unsigned long long *skip_count, void *stream, const blasst_opts *opts) {
     return run_decode(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
                       opts, false);
+}
+
+blasst_status blasst_decode_fp8(const void *q, const void *k8, const void *v8, void *o, float *lse, int B, int Hq,
+                               int Hkv, int Lq, int Lk, int d, float scale, float k_scale, float v_scale,
+                               float lambda, int causal, uint32_t *skip_mask, unsigned long long *skip_count,
+                               void *stream, const blasst_opts *opts) {
+    if (!v8) return BLASST_ERR_INVALID;
+    const Fp8Cache f8{k_scale, v_scale};
+    return run_decode(q, k8, v8, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
+                      opts, false, nullptr, &f8);
 }
 
 blasst_status blasst_decode_paged(const void *q, const void *k_pages, const void *v_pages, void *o,

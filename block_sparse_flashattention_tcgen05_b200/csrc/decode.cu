@@ -28,6 +28,7 @@
 // ring, no decision, no V) and has no forced first block.  Scores are handled
 // in log2 units: s2 = (q.k) * scale * log2(e), compared with log2(lambda).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "internal.h"
@@ -57,9 +58,37 @@ struct DecodeSmemTail {
     int abort;
 };
 
-template <int NK, int NV, bool CALIB>
+// FP8 K/V cache: a ring stage is one 128-byte-swizzled box of 64 keys x 128 e4m3 bytes, and each
+// consumer warp converts its 16 keys to f16 in a private slice laid out like a bf16 tile's 16 rows
+// (two 64-column boxes of 16 rows x 128 bytes), one slice for K and one for V.
+constexpr int kStageBytesF8 = kDecodeBlockN * 128;
+constexpr int kSliceBoxBytes = 16 * 128;
+constexpr int kSliceBytes = 2 * kSliceBoxBytes;
+
+template <int NK, int NV, bool CALIB, bool F8>
 constexpr int decode_smem_bytes() {
-    return NK * kStageBytes + (CALIB ? 0 : NV * kStageBytes) + (int)sizeof(DecodeSmemTail) + kMaxBlocksPerSplit + 1024;
+    return (NK + (CALIB ? 0 : NV)) * (F8 ? kStageBytesF8 : kStageBytes) + (F8 ? 2 * kConsumerWarps * kSliceBytes : 0) +
+           (int)sizeof(DecodeSmemTail) + kMaxBlocksPerSplit + 1024;
+}
+
+// Warp `warp`'s 16 keys of a TMA-staged e4m3 block -> f16 in its slice (see kSliceBytes).
+// Lane: row lane/2 of the 16, 64 of the 128 columns.
+__device__ __forceinline__ void convert_slice_f8(const uint8_t *stage, uint8_t *slice, int warp, int lane) {
+    const int r = lane >> 1, h = lane & 1;
+    const uint8_t *src = stage + (warp * 16 + r) * 128;
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        const int c8 = h * 4 + c;  // 16-byte chunk of e4m3: columns 16*c8 .. 16*c8 + 15
+        const uint4 v = *reinterpret_cast<const uint4 *>(src + ((c8 ^ (r & 7)) << 4));
+        uint4 a, b;
+        e4m3x4_to_f16x4(v.x, a.x, a.y);
+        e4m3x4_to_f16x4(v.y, a.z, a.w);
+        e4m3x4_to_f16x4(v.z, b.x, b.y);
+        e4m3x4_to_f16x4(v.w, b.z, b.w);
+        const int f0 = 2 * c8, f1 = 2 * c8 + 1;  // 16-byte chunks of f16
+        *reinterpret_cast<uint4 *>(slice + (f0 >> 3) * kSliceBoxBytes + swz128(r, f0 & 7)) = a;
+        *reinterpret_cast<uint4 *>(slice + (f1 >> 3) * kSliceBoxBytes + swz128(r, f1 & 7)) = b;
+    }
 }
 
 __device__ __forceinline__ void set_timeout(DecodeSmemTail *t, unsigned int *status) {
@@ -80,15 +109,17 @@ __device__ __forceinline__ int2 kv_block_coord(const DecodeParams &p, int b, int
     return make_int2(0, page * p.Hkv + hkv);
 }
 
-template <int NT, int NK, int NV, bool CALIB>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NT, int NK, int NV, bool CALIB, bool F8>
+__global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
     decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kring = smem;
-    uint8_t *vring = smem + NK * kStageBytes;
-    DecodeSmemTail *tl = reinterpret_cast<DecodeSmemTail *>(vring + (CALIB ? 0 : NV * kStageBytes));
+    constexpr int SB = F8 ? kStageBytesF8 : kStageBytes;  // bytes of one K or V ring stage
+    uint8_t *vring = smem + NK * SB;
+    uint8_t *slices = vring + (CALIB ? 0 : NV * SB);  // FP8: per consumer warp, a K and a V slice
+    DecodeSmemTail *tl = reinterpret_cast<DecodeSmemTail *>(slices + (F8 ? 2 * kConsumerWarps * kSliceBytes : 0));
     volatile uint8_t *dec = reinterpret_cast<volatile uint8_t *>(tl + 1);
 
     // CTA order: every (sequence, KV head)'s first split, then its last split, then the middle ones.
@@ -163,10 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int blk = (seed && e == 0) ? 0 : j0 + e - seed;
             const int2 cr = kv_block_coord(p, b, hkv, blk);
-            uint8_t *dst = kring + slot * kStageBytes;
-            mbar_arrive_expect_tx(&tl->k_full[slot], kStageBytes);
+            uint8_t *dst = kring + slot * SB;
+            mbar_arrive_expect_tx(&tl->k_full[slot], SB);
             tma_load_3d(dst, &tmap_k, &tl->k_full[slot], 0, cr.x, cr.y);
-            tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, cr.x, cr.y);
+            if (!F8) tma_load_3d(dst + kBoxBytes, &tmap_k, &tl->k_full[slot], 64, cr.x, cr.y);
             issued++;
         }
         if (tl->abort) {  // let copies in flight land before the CTA exits
@@ -196,10 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const int2 cr = kv_block_coord(p, b, hkv, j0 + jj);
-            uint8_t *dst = vring + slot * kStageBytes;
-            mbar_arrive_expect_tx(&tl->v_full[slot], kStageBytes);
+            uint8_t *dst = vring + slot * SB;
+            mbar_arrive_expect_tx(&tl->v_full[slot], SB);
             tma_load_3d(dst, &tmap_v, &tl->v_full[slot], 0, cr.x, cr.y);
-            tma_load_3d(dst + kBoxBytes, &tmap_v, &tl->v_full[slot], 64, cr.x, cr.y);
+            if (!F8) tma_load_3d(dst + kBoxBytes, &tmap_v, &tl->v_full[slot], 64, cr.x, cr.y);
             vk++;
         }
         if (tl->abort) {
@@ -223,6 +254,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < 8; ks++) {
             qf[ks][nt][0] = n < p.R ? __ldg(qr + ks * 8 + t4) : 0u;
             qf[ks][nt][1] = n < p.R ? __ldg(qr + ks * 8 + 4 + t4) : 0u;
+            if (F8) {  // the FP8 path multiplies in f16: q re-rounded from bf16 (exact in f16's normal range)
+#pragma unroll
+                for (int u = 0; u < 2; u++)
+                    qf[ks][nt][u] = pack_f16x2(__uint_as_float(qf[ks][nt][u] << 16),
+                                               __uint_as_float(qf[ks][nt][u] & 0xFFFF0000u));
+            }
         }
     }
     // last visible key of each of my columns (col = nt*8 + 2*t4 + e)
@@ -290,17 +327,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pv[2 + e2] = hs[nt][2 + e2] == NEG_INF ? 0.f : ex2(hs[nt][2 + e2] - mnew);
                 lsum[nt][e2] += pv[e2] + pv[2 + e2];
             }
-            const uint32_t lo = pack_bf16x2(pv[0], pv[1]);
-            const uint32_t hi = pack_bf16x2(pv[2], pv[3]);
-            lrnd[nt][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
-            lrnd[nt][1] += __uint_as_float(lo & 0xFFFF0000u) + __uint_as_float(hi & 0xFFFF0000u);
+            uint32_t lo, hi;
+            if constexpr (F8) {
+                lo = pack_f16x2(pv[0], pv[1]);
+                hi = pack_f16x2(pv[2], pv[3]);
+                const float2 l2 = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+                const float2 h2 = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+                lrnd[nt][0] += l2.x + h2.x;
+                lrnd[nt][1] += l2.y + h2.y;
+            } else {
+                lo = pack_bf16x2(pv[0], pv[1]);
+                hi = pack_bf16x2(pv[2], pv[3]);
+                lrnd[nt][0] += __uint_as_float(lo << 16) + __uint_as_float(hi << 16);
+                lrnd[nt][1] += __uint_as_float(lo & 0xFFFF0000u) + __uint_as_float(hi & 0xFFFF0000u);
+            }
             pb[nt][0] = movmatrix_t(lo);
             pb[nt][1] = movmatrix_t(hi);
         }
         const int vslot = kept_count % NV;
         if (!mbar_wait(&tl->v_full[vslot], (kept_count / NV) & 1, &tl->abort)) set_timeout(tl, p.status);
-        const uint8_t *vb = vring + vslot * kStageBytes;
-        {
+        const uint8_t *vb = vring + vslot * SB;
+        if constexpr (F8) {
+            uint8_t *vs = slices + (kConsumerWarps + warp) * kSliceBytes;
+            __syncwarp();  // the previous block's ldmatrix reads of this slice are done
+            convert_slice_f8(vb, vs, warp, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->v_empty[vslot]);  // the stage is free once converted
+            const int mi = lane >> 3, ri = lane & 7;
+            const int r = ri + 8 * (mi >> 1);
+#pragma unroll
+            for (int mt = 0; mt < 8; mt++) {
+                const int chunk = mt * 2 + (mi & 1);
+                uint32_t a[4];
+                ldsm_x4_t(smem_addr(vs + (chunk >> 3) * kSliceBoxBytes + swz128(r, chunk & 7)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) mma_f16_16816(o_acc[mt][nt], a, pb[nt]);
+            }
+        } else {
             const int mi = lane >> 3, ri = lane & 7;
             const int key = warp * 16 + ri + 8 * (mi >> 1);
 #pragma unroll
@@ -311,9 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int nt = 0; nt < NT; nt++) mma_bf16_16816(o_acc[mt][nt], a, pb[nt]);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->v_empty[vslot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tl->v_empty[vslot]);
         kept_count++;
     };
     // queue a decided block, and run P.V for the oldest one if it was kept
@@ -363,12 +426,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = jj < 0 ? 0 : j0 + jj;
         const int slot = e % NK;
         if (!mbar_wait(&tl->k_full[slot], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
-        const uint8_t *kb = kring + slot * kStageBytes;
+        const uint8_t *kb = kring + slot * SB;
 
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        {
+        if constexpr (F8) {
+            uint8_t *ks_ = slices + warp * kSliceBytes;
+            __syncwarp();  // the previous block's ldmatrix reads of this slice are done
+            convert_slice_f8(kb, ks_, warp, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->k_empty[slot]);  // the stage is free once converted
+            const int mi = lane >> 3, ri = lane & 7;
+            const int r = ri + 8 * (mi & 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++) {
+                const int chunk = ks * 2 + (mi >> 1);
+                uint32_t a[4];
+                ldsm_x4(smem_addr(ks_ + (chunk >> 3) * kSliceBoxBytes + swz128(r, chunk & 7)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) mma_f16_16816(acc[nt], a, qf[ks][nt]);
+            }
+        } else {
             const int mi = lane >> 3, ri = lane & 7;
             const int key = warp * 16 + ri + 8 * (mi & 1);
 #pragma unroll
@@ -379,9 +458,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int nt = 0; nt < NT; nt++) mma_bf16_16816(acc[nt], a, qf[ks][nt]);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->k_empty[slot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tl->k_empty[slot]);
 
         // scaled, masked scores in log2 units; my keys: lo = g4, hi = g4 + 8
         const int key_lo = j * kDecodeBlockN + warp * 16 + g4;
@@ -555,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             o += obuf[(w * 128 + x) * NC + c];
         }
         const size_t row = (size_t)(qrow0 + c) * S + split;
-        p.part_o[row * 128 + x] = lr > 0.f ? o / lr : 0.f;
+        p.part_o[row * 128 + x] = lr > 0.f ? (F8 ? p.v_scale : 1.f) * o / lr : 0.f;
         if (x == 0) p.part_lse[row] = l > 0.f ? (tl->mfin[c] + __log2f(l)) * 0.69314718055994531f : NEG_INF;
     }
 }
@@ -599,11 +678,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
     if (lane == 0) p.lse[row] = L;
 }
 
-template <int NT, bool CALIB>
+template <int NT, bool CALIB, bool F8 = false>
 cudaError_t launch_decode_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st) {
     constexpr int NK = 4, NV = 2;
-    constexpr int smem = decode_smem_bytes<NK, NV, CALIB>();
-    auto kern = decode_split_kernel<NT, NK, NV, CALIB>;
+    constexpr int smem = decode_smem_bytes<NK, NV, CALIB, F8>();
+    auto kern = decode_split_kernel<NT, NK, NV, CALIB, F8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<p.num_splits * p.Hkv * p.B, kThreads, smem, st>>>(p, tk, tv);
@@ -616,6 +695,11 @@ cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tk, const CU
                           cudaStream_t st) {
     if (calib) return nt == 1 ? launch_decode_t<1, true>(p, tk, tv, st) : launch_decode_t<2, true>(p, tk, tv, st);
     return nt == 1 ? launch_decode_t<1, false>(p, tk, tv, st) : launch_decode_t<2, false>(p, tk, tv, st);
+}
+
+cudaError_t launch_decode_fp8(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int nt,
+                              cudaStream_t st) {
+    return nt == 1 ? launch_decode_t<1, false, true>(p, tk, tv, st) : launch_decode_t<2, false, true>(p, tk, tv, st);
 }
 
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t st) {

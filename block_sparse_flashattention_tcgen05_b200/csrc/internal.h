@@ -27,6 +27,7 @@ struct DecodeParams {
     float scale_log2;               // scale * log2(e)
     float thr_log2;                 // log2(lambda), -inf for lambda = 0
     int seed;                       // 1: splits after the first start from block 0's row maxima
+    float v_scale;                  // FP8 cache: V = v_scale * e4m3 (scale_log2 already holds k_scale)
     // paged cache (null: contiguous): K/V pages [num_pages, Hkv, 64, 128]; sequence b has
     // seq_lens[b] keys in pages block_table[b * nb + i]; Lk and nb are then the maxima
     const int *block_table;
@@ -100,6 +101,9 @@ void set_last_error(const char *msg);
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
                           int nt, cudaStream_t stream);
+// FP8 (e4m3) K/V cache, d = 128, tiles of up to 16 rows; tmaps are u8 boxes of 128 x 64
+cudaError_t launch_decode_fp8(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, int nt,
+                              cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t stream);
 // Decode tiles of 17..128 rows (d = 128) on tcgen05; tmap_q covers q as [B][Hq*Lq][128].
 cudaError_t launch_decode_wide(const DecodeParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,

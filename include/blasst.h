@@ -136,6 +136,29 @@ BLASST_API blasst_status blasst_decode(const void *q, const void *k, const void 
                             void *stream, const blasst_opts *opts);
 
 /*
+ * Decode over an FP8 (e4m3, OCP "E4M3FN": bias 7, no infinities) KV cache.
+ * Not on the pages: a storage format that halves the bytes of K and V, which
+ * decode reads from HBM once per step.  The cache holds K = k_scale * k8 and
+ * V = v_scale * v8 (per-tensor scales, finite and > 0); the arithmetic is
+ * exactly blasst_decode's on those dequantized values (same tile, 64-key
+ * blocks, splits, skip rule, combine), with one difference in rounding: the
+ * products run in f16 (e4m3 -> f16 is exact; q is re-rounded from bf16 to
+ * f16, which is exact for |q| in f16's normal range, 6.1e-5 .. 65504; P is
+ * rounded to f16 before P.V).
+ *
+ * k8, v8  [B, Hkv, Lk, 128] bytes (e4m3), 16-byte aligned, dense rows.
+ * q, o, lse, skip_mask, skip_count, stream and opts (num_splits, workspace,
+ * status_word, seed_splits) as blasst_decode.  d = 128 and G * Lq <= 16 only
+ * (BLASST_ERR_UNSUPPORTED otherwise); non-finite or non-positive scales are
+ * BLASST_ERR_INVALID.
+ */
+BLASST_API blasst_status blasst_decode_fp8(const void *q, const void *k8, const void *v8, void *o, float *lse,
+                                           int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                                           float k_scale, float v_scale, float lambda, int causal,
+                                           uint32_t *skip_mask, unsigned long long *skip_count, void *stream,
+                                           const blasst_opts *opts);
+
+/*
  * Decode over a paged, ragged KV cache.  Not on the pages as such: they report
  * the method integrated into serving frameworks (xllm-io paper review,
  * overview table; gist.science (de), section 1), whose caches are paged.  Per

@@ -52,6 +52,8 @@ __all__ = [
     "planted_decode",
     "planted_mla",
     "upstream_grad",
+    "e4m3_bits",
+    "e4m3_to_f32",
 ]
 
 _TENSOR_ID = {"q": 1, "k": 2, "v": 3, "u": 4, "w": 5, "h": 6, "do": 7}
@@ -303,3 +305,23 @@ def upstream_grad(B, Hq, Lq, dv=128, seed=0) -> np.ndarray:
     do = np.empty((B, Hq, Lq, dv), np.uint16)
     _fill(do, seed, _TENSOR_ID["do"])
     return do
+
+
+def e4m3_to_f32(b: np.ndarray) -> np.ndarray:
+    """e4m3 bytes (OCP E4M3FN: sign, 4-bit exponent with bias 7, 3-bit mantissa, no
+    infinities, S.1111.111 = NaN) -> float32 values, exactly."""
+    b = np.asarray(b, dtype=np.uint8).astype(np.int32)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = np.where((e == 15) & ((b & 7) == 7), np.nan, val)
+    return (sign * val).astype(np.float32)
+
+
+def e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """float values -> e4m3 bytes, round to nearest even, saturated at +-448 (torch's cast)."""
+    import torch
+
+    x = np.clip(np.asarray(x, dtype=np.float32), -448.0, 448.0)
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()

@@ -149,6 +149,26 @@ def test_backward_workspace_bytes(bl):
     assert f(0, 1, 1) == 0 and f(1, 1, 0) == 0
 
 
+def _fp8(bl, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=8, Hkv=1, Lq=1, Lk=256, d=128, scale=0.088,
+             ks=0.01, vs=0.01, lam=0.0, causal=0)
+    a.update(over)
+    return bl.lib().blasst_decode_fp8(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Lq"],
+                                      a["Lk"], a["d"], a["scale"], a["ks"], a["vs"], a["lam"], a["causal"], None,
+                                      None, None, ctypes.byref(a.get("opts") or bl.Opts()))
+
+
+def test_fp8_decode_arguments_rejected_before_launch(bl):
+    assert _fp8(bl, v=None) == 1
+    assert _fp8(bl, k=FAKE + 8) == 1
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert _fp8(bl, ks=bad) == 1 and _fp8(bl, vs=bad) == 1
+    assert _fp8(bl, d=64) == 2
+    assert _fp8(bl, Hq=32) == 2                      # more than 16 rows per tile
+    assert _fp8(bl, opts=bl.Opts(k_row_stride=256)) == 2
+    assert _fp8(bl, lam=1.0) == 1
+
+
 def test_calibrate_requires_gaps_and_valid_mode(bl):
     assert _call(bl, "blasst_calibrate") == 1                 # no gaps_out
     assert _call(bl, "blasst_calibrate", opts=bl.Opts(mode=7, gaps_out=FAKE)) == 1

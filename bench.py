@@ -380,6 +380,55 @@ class DecodeSeeded(Decode):
     seed_splits = True
 
 
+class DecodeFp8(Decode):
+    """The batch-32 GQA decode over an FP8 (e4m3) copy of the same cache, per-tensor
+    scales (max |x| / 448), quantised on the device.  Effective bytes: all K bytes
+    (1 per element), kept V blocks (8 KiB each), q and o.  λ: the bf16 decode's
+    calibration (the sweep reports the sparsity each λ reaches here)."""
+
+    kind = "decode_fp8"
+
+    def __init__(self, src, device):
+        import torch
+
+        self.__dict__.update(src.__dict__)
+        self.cfg = dict(src.cfg, workload=src.cfg["workload"] + ", FP8 (e4m3) K/V cache")
+
+        def quant(x):
+            sc = float(x.float().abs().max().item()) / 448.0
+            return (x.float() / sc).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8), sc
+
+        self.k8, self.k_scale = quant(src.k)
+        self.v8, self.v_scale = quant(src.v)
+        self.launches = 2
+
+    def call(self, lam, stream=None):
+        return self.bl.decode_fp8(self.q, self.k8, self.v8, scale=self.inp.scale, k_scale=self.k_scale,
+                                  v_scale=self.v_scale, lam=lam, num_splits=self.cfg["splits"], o=self.o,
+                                  lse=self.lse, skip_mask=False, skip_count=self.count, workspace=self.ws,
+                                  stream=stream)
+
+    def work(self, skipped):
+        c = self.cfg
+        kept = self.visited - skipped
+        qo = self.inp.q.nbytes * 2 + self.lse.numel() * 4
+        return c["B"] * c["Hkv"] * c["Lk"] * c["d"] + kept * 64 * c["d"] + qo
+
+    def host_bytes(self):
+        return (self.inp.q.nbytes + self.k8.numel() + self.v8.numel(), self.inp.q.nbytes + self.lse.numel() * 4)
+
+    def e2e_call(self, lam, hq, hk, hv, ho, hl):
+        """q and the e4m3 cache from pinned host memory, o and lse back."""
+        if getattr(self, "_h8", None) is None:
+            self._h8 = (self.k8.cpu().pin_memory(), self.v8.cpu().pin_memory())
+        self.q.copy_(hq, non_blocking=True)
+        self.k8.copy_(self._h8[0], non_blocking=True)
+        self.v8.copy_(self._h8[1], non_blocking=True)
+        self.call(lam)
+        ho.copy_(self.o, non_blocking=True)
+        hl.copy_(self.lse, non_blocking=True)
+
+
 class DecodeMqa(Decode):
     """Decode with a 128-row tile (128 query heads on one KV head): the tcgen05 kernel."""
 
@@ -849,7 +898,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     wl_kind = args.workload
-    cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2, "backward": 0}[wl_kind]]
+    cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2, "backward": 0, "decode_fp8": 1}[wl_kind]]
     per_step = []
     vals = []
     budget = float(os.environ.get("BLASST_REF_STEP_SECONDS", "8"))
@@ -880,7 +929,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--workload", choices=["prefill", "decode", "mla", "backward"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "decode", "mla", "backward", "decode_fp8"], default="prefill")
     ap.add_argument("--size", choices=sorted(SIZES), default="full",
                     help="full = the benchmark shapes; medium = profiling size; quick = smoke-testing the bench")
     ap.add_argument("--no-sweep", action="store_true")
@@ -892,6 +941,7 @@ def main():
     ap.add_argument("--no-paged", action="store_true", help="skip the paged, ragged decode rows of the sweep")
     ap.add_argument("--no-mqa", action="store_true", help="skip the 128-head MQA decode rows of the sweep")
     ap.add_argument("--no-backward", action="store_true", help="skip the fixed-mask backward rows of the sweep")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-cache decode rows of the sweep")
     ap.add_argument("--calibration", action="store_true",
                     help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
     args = ap.parse_args()
@@ -930,8 +980,10 @@ def main():
             wls.pop("prefill", None)
             notes.append("prefill kernel not available in this build; headline falls back to decode")
             headline_kind = "decode"
-    if headline_kind == "decode":
+    if headline_kind in ("decode", "decode_fp8"):
         wls["decode"] = Decode(dcfg, dev)
+    if headline_kind == "decode_fp8":
+        wls["decode_fp8"] = DecodeFp8(wls["decode"], dev)
     if headline_kind == "mla":
         wls["mla"] = Mla(mcfg, dev)
     if headline_kind == "backward":
@@ -991,6 +1043,8 @@ def main():
             ws = DecodeSeeded.__new__(DecodeSeeded)  # shares the decode workload's inputs and buffers
             ws.__dict__.update(wls["decode"].__dict__)
             wls["decode_seeded"] = ws
+        if not args.no_fp8:
+            wls["decode_fp8"] = DecodeFp8(wls["decode"], dev)
         if not args.no_paged:
             wls["decode_paged"] = DecodePaged(wls["decode"], dev,
                                               min_len=min(8192, wls["decode"].cfg["Lk"] // 4))
@@ -1005,6 +1059,8 @@ def main():
             wls["prefill_64k"] = Prefill(PREFILL_64K, dev)
         if "backward" in wls and "prefill" in lams and "backward" not in lams:
             lams["backward"] = lams["prefill"]  # same inputs, same forward masks
+        if "decode_fp8" in wls and "decode" in lams and "decode_fp8" not in lams:
+            lams["decode_fp8"] = lams["decode"]
         for k, w in wls.items():
             if k not in lams:
                 lams[k] = w.lambdas() if hasattr(w, "lambdas") else lambdas_for_targets(w, w.calibrate())

@@ -60,14 +60,15 @@ struct DecodeSmemTail {
 
 // FP8 K/V cache: a ring stage is one 128-byte-swizzled box of 64 keys x 128 e4m3 bytes, and each
 // consumer warp converts its 16 keys to f16 in a private slice laid out like a bf16 tile's 16 rows
-// (two 64-column boxes of 16 rows x 128 bytes), one slice for K and one for V.
+// (two 64-column boxes of 16 rows x 128 bytes): two K slices (block j+1 is converted while the
+// warps meet for block j's decision) and one V slice.
 constexpr int kStageBytesF8 = kDecodeBlockN * 128;
 constexpr int kSliceBoxBytes = 16 * 128;
 constexpr int kSliceBytes = 2 * kSliceBoxBytes;
 
 template <int NK, int NV, bool CALIB, bool F8>
 constexpr int decode_smem_bytes() {
-    return (NK + (CALIB ? 0 : NV)) * (F8 ? kStageBytesF8 : kStageBytes) + (F8 ? 2 * kConsumerWarps * kSliceBytes : 0) +
+    return (NK + (CALIB ? 0 : NV)) * (F8 ? kStageBytesF8 : kStageBytes) + (F8 ? 3 * kConsumerWarps * kSliceBytes : 0) +
            (int)sizeof(DecodeSmemTail) + kMaxBlocksPerSplit + 1024;
 }
 
@@ -118,8 +119,8 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
     uint8_t *kring = smem;
     constexpr int SB = F8 ? kStageBytesF8 : kStageBytes;  // bytes of one K or V ring stage
     uint8_t *vring = smem + NK * SB;
-    uint8_t *slices = vring + (CALIB ? 0 : NV * SB);  // FP8: per consumer warp, a K and a V slice
-    DecodeSmemTail *tl = reinterpret_cast<DecodeSmemTail *>(slices + (F8 ? 2 * kConsumerWarps * kSliceBytes : 0));
+    uint8_t *slices = vring + (CALIB ? 0 : NV * SB);  // FP8: per consumer warp, two K slices, then the V slices
+    DecodeSmemTail *tl = reinterpret_cast<DecodeSmemTail *>(slices + (F8 ? 3 * kConsumerWarps * kSliceBytes : 0));
     volatile uint8_t *dec = reinterpret_cast<volatile uint8_t *>(tl + 1);
 
     // CTA order: every (sequence, KV head)'s first split, then its last split, then the middle ones.
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
         if (!mbar_wait(&tl->v_full[vslot], (kept_count / NV) & 1, &tl->abort)) set_timeout(tl, p.status);
         const uint8_t *vb = vring + vslot * SB;
         if constexpr (F8) {
-            uint8_t *vs = slices + (kConsumerWarps + warp) * kSliceBytes;
+            uint8_t *vs = slices + (2 * kConsumerWarps + warp) * kSliceBytes;
             __syncwarp();  // the previous block's ldmatrix reads of this slice are done
             convert_slice_f8(vb, vs, warp, lane);
             __syncwarp();
@@ -421,22 +422,31 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
         if (hk) pv_block(hs, hmo, hmn);
     };
 
+    // FP8: K of ring entry e -> this warp's K slice e & 1, then the ring stage goes back
+    auto convert_k = [&](int e) {
+        const int ns = e % NK;
+        if (!mbar_wait(&tl->k_full[ns], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
+        __syncwarp();  // the slice's previous ldmatrix reads are done
+        convert_slice_f8(kring + ns * SB, slices + (warp * 2 + (e & 1)) * kSliceBytes, warp, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl->k_empty[ns]);
+    };
+    if constexpr (F8) {
+        if (nent > 0) convert_k(0);
+    }
+
     for (int e = 0; e < nent; e++) {
         const int jj = e - seed;  // block index within the split; -1: the seed block
         const int j = jj < 0 ? 0 : j0 + jj;
         const int slot = e % NK;
-        if (!mbar_wait(&tl->k_full[slot], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
+        if (!F8 && !mbar_wait(&tl->k_full[slot], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
         const uint8_t *kb = kring + slot * SB;
 
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         if constexpr (F8) {
-            uint8_t *ks_ = slices + warp * kSliceBytes;
-            __syncwarp();  // the previous block's ldmatrix reads of this slice are done
-            convert_slice_f8(kb, ks_, warp, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tl->k_empty[slot]);  // the stage is free once converted
+            const uint8_t *ks_ = slices + (warp * 2 + (e & 1)) * kSliceBytes;  // converted ahead
             const int mi = lane >> 3, ri = lane & 7;
             const int r = ri + 8 * (mi & 1);
 #pragma unroll
@@ -485,6 +495,9 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
                 tl->red[e & 1][warp][nt * 8 + 2 * t4] = cmax[nt][0];
                 tl->red[e & 1][warp][nt * 8 + 2 * t4 + 1] = cmax[nt][1];
             }
+        }
+        if constexpr (F8) {
+            if (e + 1 < nent) convert_k(e + 1);  // overlaps the other warps reaching the barrier
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 

@@ -13,7 +13,7 @@ import os
 __all__ = [
     "BlasstError", "lib", "prefill", "decode", "decode_noalloc", "calibrate", "calibrate_fit", "calibrate_threshold",
     "visited_pairs", "decode_workspace_bytes", "mask_words", "Opts", "STATUS", "prefill_backward",
-    "backward_workspace_bytes", "decode_fp8",
+    "backward_workspace_bytes", "decode_fp8", "decode_pick_splits",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.blasst_calibrate_threshold.restype = ctypes.c_int
         L.blasst_calibrate_threshold.argtypes = [ctypes.c_void_p, ctypes.c_longlong, ctypes.c_double,
                                                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+        L.blasst_decode_pick_splits.restype = ctypes.c_int
+        L.blasst_decode_pick_splits.argtypes = [ctypes.c_int] * 4
         L.blasst_decode_workspace_bytes.restype = ctypes.c_size_t
         L.blasst_decode_workspace_bytes.argtypes = [ctypes.c_int] * 5
         L.blasst_visited_pairs.restype = ctypes.c_longlong
@@ -212,6 +214,15 @@ def prefill_backward(q, k, v, o, lse, dout, *, scale, causal=True, skip_mask=Non
                                        _ptr(skip_mask), _stream(stream), ctypes.byref(opts))
     _check(rc, "blasst_prefill_backward")
     return dq, dk, dv
+
+
+def decode_pick_splits(B, Hkv, Lk, num_sms=None) -> int:
+    """The split count num_splits=-1 selects (num_sms: this device's SM count by default)."""
+    if num_sms is None:
+        import torch
+
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return int(lib().blasst_decode_pick_splits(B, Hkv, Lk, num_sms))
 
 
 def backward_workspace_bytes(B, Hq, Lq) -> int:

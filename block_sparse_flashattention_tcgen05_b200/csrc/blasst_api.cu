@@ -256,11 +256,17 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     const bool wide = R > 16;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
     if (wide && op.seed_splits) return BLASST_ERR_UNSUPPORTED;
-    if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + (op.num_splits ? op.num_splits : 16) - 1) /
-                        (op.num_splits ? op.num_splits : 16) > 1024)
-        return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 blocks per split
-    const int S = op.num_splits ? op.num_splits : 16;
+    int S = op.num_splits ? op.num_splits : 16;
+    if (S == -1) {  // adaptive: from the batch, the cache length and this device's SM count
+        int dev = 0, sms = 0;
+        cudaError_t ed = cudaGetDevice(&dev);
+        if (ed == cudaSuccess) ed = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (ed != cudaSuccess) return cuda_fail(ed, "cudaDeviceGetAttribute(multiprocessors)");
+        S = blasst_decode_pick_splits(B, Hkv, Lk, sms);
+    }
     if (S < 1 || S > 65535) return BLASST_ERR_INVALID;
+    if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + S - 1) / S > 1024)
+        return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 blocks per split
     if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;
     const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
     const int per_split = (nb + S - 1) / S;
@@ -618,6 +624,15 @@ blasst_status blasst_calibrate_threshold(const float *gaps, long long n, double 
     *lambda_out = lam;
     if (achieved_out) *achieved_out = n_vis ? (double)got / (double)n_vis : 0.0;
     return BLASST_OK;
+}
+
+int blasst_decode_pick_splits(int B, int Hkv, int Lk, int num_sms) {
+    if (B <= 0 || Hkv <= 0 || Lk <= 0 || num_sms <= 0) return 1;
+    const long long groups = (long long)B * Hkv;
+    const long long nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
+    const long long cap = std::max(1LL, std::min(64LL, nb / 32));  // at least 32 blocks per split
+    const long long want = (16LL * num_sms + groups - 1) / groups;  // about 16 CTAs per SM over the call
+    return (int)std::max(1LL, std::min(cap, want));
 }
 
 size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_splits) {

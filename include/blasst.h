@@ -82,7 +82,10 @@ typedef struct blasst_opts {
     size_t struct_size;
     int dv;                    /* value head dim; 0 -> d.  MLA: d = 576, dv = 512 */
     int block_n;               /* 0, or the fixed block size (128 prefill, 64 decode) */
-    int num_splits;            /* decode: KV chunks per sequence; 0 -> 16 */
+    int num_splits;            /* decode: KV chunks per sequence; 0 -> 16; -1 -> adaptive
+                                  (blasst_decode, _decode_paged, _decode_fp8 with d = 128:
+                                  blasst_decode_pick_splits with this device's SM count;
+                                  MLA and the no-allocation call reject it) */
     int mode;                  /* blasst_calibrate only: 0 = prefill tiling, 1 = decode tiling */
     long long k_row_stride;    /* elements between consecutive keys; 0 -> d */
     long long v_row_stride;    /* elements between consecutive values; 0 -> dv */
@@ -286,6 +289,18 @@ BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, con
                                                const blasst_opts *opts);
 
 /* Bytes of decode workspace for these sizes (num_splits 0 -> 16, dv 0 -> 128). */
+/* Host only.  The split count that num_splits = -1 selects for a decode of B
+ * sequences x Hkv KV heads over Lk keys on a device with num_sms SMs: about
+ * 16 CTAs per SM over the call (ceil(16 * num_sms / (B * Hkv))), but at least
+ * 32 blocks of 64 keys per split, and at most 64 splits; 1 for short caches.
+ * Not on the pages (split-KV is not); it follows a measured sweep on B200:
+ * batch 32 x 8 KV heads at 32K keys is as fast at 8-16 splits as at any count
+ * and loses reachable sparsity past 16, while batch 1 needs 16-32 to fill the
+ * device.  A decode that used -1 is reproduced by passing this count
+ * explicitly (the skip mask depends on the split count).  Size a caller
+ * workspace with it too.  Invalid sizes return 1. */
+BLASST_API int blasst_decode_pick_splits(int B, int Hkv, int Lk, int num_sms);
+
 BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_splits);
 
 /* Number of visited (tile, block) pairs: the sparsity denominator.

@@ -169,6 +169,27 @@ def test_fp8_decode_arguments_rejected_before_launch(bl):
     assert _fp8(bl, lam=1.0) == 1
 
 
+def test_pick_splits(bl):
+    f = bl.lib().blasst_decode_pick_splits
+    assert f(32, 8, 32768, 148) == 10       # ceil(16 * 148 / 256)
+    assert f(1, 8, 32768, 148) == 16        # capped at 32 blocks (2048 keys) per split
+    assert f(4, 8, 32768, 148) == 16
+    assert f(1, 1, 1 << 20, 148) == 64      # never more than 64
+    assert f(1, 8, 2047, 148) == 1          # short cache: one split
+    assert f(4096, 8, 32768, 148) == 1      # large batch fills the device by itself
+    for B in (1, 2, 8, 64, 512):
+        s = f(B, 8, 65536, 132)
+        assert 1 <= s <= max(1, 1024 // 32) and s == max(1, min(min(64, 1024 // 32), -(-16 * 132 // (B * 8))))
+    assert f(0, 8, 100, 148) == 1 and f(1, 8, 100, 0) == 1
+
+
+def test_adaptive_splits_only_where_supported(bl):
+    mla = dict(num_splits=-1, dv=512, k_row_stride=576, v_row_stride=576)
+    assert _call(bl, "blasst_decode", d=576, opts=bl.Opts(**mla)) == 1   # MLA
+    assert _call(bl, "blasst_decode_noalloc", opts=bl.Opts(num_splits=-1)) == 1
+    assert _call(bl, "blasst_decode", opts=bl.Opts(num_splits=-2)) == 1
+
+
 def test_calibrate_requires_gaps_and_valid_mode(bl):
     assert _call(bl, "blasst_calibrate") == 1                 # no gaps_out
     assert _call(bl, "blasst_calibrate", opts=bl.Opts(mode=7, gaps_out=FAKE)) == 1

@@ -307,3 +307,16 @@ def test_decode_full_size_sampled(bl, lam):
     rng = np.random.default_rng(0)
     tiles = np.sort(rng.choice(32 * 8, 12, replace=False))
     check_decode(bl, inp, lam, False, 16, tiles=tiles)
+
+
+def test_decode_adaptive_splits(bl):
+    # num_splits=-1 picks blasst_decode_pick_splits(B, Hkv, Lk, SMs); same bytes as passing that count
+    inp = planted_decode(2, 8, 2, 64 * 300 + 5, 128, seed=29, reading="blk")
+    S = bl.decode_pick_splits(2, 2, 64 * 300 + 5)
+    assert S == max(1, min(64, 300 // 32, -(-16 * torch.cuda.get_device_properties(0).multi_processor_count // 4)))
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    a = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=-1)
+    b = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=S)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    check_decode(bl, inp, 0.05, False, S)

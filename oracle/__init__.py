@@ -264,3 +264,52 @@ def attention_backward(q, k, v, do, *, scale, causal, skip=None, BM=BM_PREFILL, 
             dq[b, h] = scale * (dS @ K[b, hk])
             dk[b, hk] += scale * (dS.T @ Q[b, h])
     return dict(dq=dq, dk=dk, dv=dvv, o=o, lse=lse)
+
+
+def backward_dq_rows(q, k, v, do, rows, *, scale, causal, skip, BM=BM_PREFILL, BN=BN_PREFILL, terms=False):
+    """dQ of chosen query rows of the fixed-mask backward, each row on its own.
+
+    A row's gradient needs only that row: its kept, visible scores S_c = scale
+    q_r . k_c, its own lse over them, P = exp(S - lse), dP_c = dO_r . v_c,
+    D = sum_c P_c dP_c, and dQ_r = scale * sum_c P_c (dP_c - D) k_c -- the same
+    definition as attention_backward, restricted to one row (O(Lk * d) work),
+    so it can be run at sizes where the whole matrix does not fit.
+    rows: iterable of (b, hq, r).  skip as in attention_backward (None: dense).
+    Returns float64 [len(rows), d]; with terms=True a dict with that ("dq") and,
+    per row, the row's P and dS over all keys ([len(rows), Lk]) and O = P V
+    ([len(rows), dv]), for tolerance models built from the same definition.
+    """
+    Q, K, V, dO = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, Hq, Lq, d = Q.shape
+    Hkv, Lk = K.shape[1], K.shape[2]
+    G = Hq // Hkv
+    nq = (Lq + BM - 1) // BM
+    nb = (Lk + BN - 1) // BN
+    if skip is not None:
+        skip = np.asarray(skip, dtype=np.uint8).reshape(B, Hq, nq, nb)
+    cols = np.arange(Lk)
+    out = np.zeros((len(rows), d))
+    Ps = np.zeros((len(rows), Lk))
+    dSs = np.zeros((len(rows), Lk))
+    Os = np.zeros((len(rows), V.shape[3]))
+    for n, (b, h, r) in enumerate(rows):
+        hk = h // G
+        keep = np.ones(Lk, bool)
+        if causal:
+            keep &= cols <= r + (Lk - Lq)
+        if skip is not None:
+            keep &= ~skip[b, h, r // BM][cols // BN].astype(bool)
+        if not keep.any():
+            continue
+        s = scale * (K[b, hk] @ Q[b, h, r])
+        m = s[keep].max()
+        e = np.where(keep, np.exp(np.where(keep, s, m) - m), 0.0)
+        p = e / e.sum()
+        dp = V[b, hk] @ dO[b, h, r]
+        dd = (p * dp).sum()
+        ds = p * (dp - dd)
+        out[n] = scale * (ds @ K[b, hk])
+        Ps[n], dSs[n], Os[n] = p, ds, p @ V[b, hk]
+    if terms:
+        return dict(dq=out, P=Ps, dS=dSs, O=Os)
+    return out

@@ -16,7 +16,7 @@ import pytest
 
 import oracle
 from _parity import bf16_tensor_to_f64, unpack_mask
-from synth import planted_prefill, random_normal, upstream_grad
+from synth import bf16_to_f32, planted_prefill, random_normal, upstream_grad
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -149,3 +149,54 @@ def test_backward_caller_workspace(bl):
     b = bl.prefill_backward(q, k, v, o, lse, do, scale=inp.scale, causal=True, skip_mask=mask)
     torch.cuda.synchronize()
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+def test_backward_full_size_sampled_rows_and_invariants(bl):
+    """The benchmark's 32K GQA shape (B=1, Hq=32, Hkv=8, causal): dq of sampled rows against the
+    oracle row by row, and, over every key, the two sums the gradient fixes at any size:
+    sum_k dK_k = 0 (softmax does not change when every key moves by the same vector) and
+    sum_k dV_k = sum of the group's dO rows (each row's P sums to 1)."""
+    L = 32768
+    inp = planted_prefill(1, 32, 8, L, 128, seed=3, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    o, lse, mask, cnt = bl.prefill(q, k, v, scale=inp.scale, lam=0.0128, causal=True)
+    do_bits = upstream_grad(1, 32, L, 128, seed=9)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv = bl.prefill_backward(q, k, v, o, lse, to_dev(do_bits), scale=inp.scale, causal=True,
+                                     skip_mask=mask, status_word=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    bits = unpack_mask(mask.cpu().numpy(), L // 128)
+    assert 0.3 < bits.sum() / bl.visited_pairs(1, 32, 8, L, L, True, False) < 0.95
+    rows = [(0, 0, 0), (0, 5, 127), (0, 9, 12345), (0, 17, 20000), (0, 26, 30001), (0, 31, L - 1)]
+    ref = oracle.backward_dq_rows(inp.q, inp.k, inp.v, do_bits, rows, scale=inp.scale, causal=True, skip=bits,
+                                  terms=True)
+    dqh = dq.float().cpu().numpy()
+    got = np.stack([dqh[b, h, r] for b, h, r in rows])
+    # A full-size row sums dS_k K_k over up to 32K keys while dq itself cancels (sum_k dS_k = 0), so
+    # the bound is per element, from the terms of those sums (worst case, no cancellation of errors):
+    #   dS_k is rounded to bf16:            2^-9 scale sum_k |dS_k K_kd|
+    #   D = rowsum(dO O) uses the forward's bf16 O, normalised by the sum of the bf16-rounded P it used,
+    #   so |dO| (2^-8 sum_k P_k |V_k| + 2^-9 |O|) bounds D's error dD, which moves dq by at most
+    #                                       scale dD sum_k P_k |K_kd|
+    #   the output is rounded to bf16:      2^-9 |dq|
+    Kf = bf16_to_f32(inp.k).astype(np.float64)[0]
+    Vf = bf16_to_f32(inp.v).astype(np.float64)[0]
+    Dof = bf16_to_f32(do_bits).astype(np.float64)[0]
+    for n, (b, h, r) in enumerate(rows):
+        kk, vv = Kf[h // 4], Vf[h // 4]
+        p_, ds_, o_ = ref["P"][n], ref["dS"][n], ref["O"][n]
+        dD = (np.abs(Dof[h, r]) * (2.0 ** -8 * (p_ @ np.abs(vv)) + 2.0 ** -9 * np.abs(o_))).sum()
+        bound = (2.0 ** -9 * (np.abs(ref["dq"][n]) + inp.scale * (np.abs(ds_) @ np.abs(kk))) +
+                 inp.scale * dD * (p_ @ np.abs(kk)))
+        err = np.abs(got[n] - ref["dq"][n])
+        assert np.all(err <= bound + 1e-7), f"row {(b, h, r)}: worst {np.max(err / (bound + 1e-7)):.2f} of bound"
+    dkh = dk.double().cpu().numpy()[0]
+    dvh = dv.double().cpu().numpy()[0]
+    dov = torch.from_numpy(do_bits.view(np.int16)).view(torch.bfloat16).double().numpy()[0]
+    for hk in range(8):
+        tot = np.abs(dkh[hk]).sum(axis=0)
+        assert np.all(np.abs(dkh[hk].sum(axis=0)) <= 2.0 ** -6 * tot)
+        want = dov[hk * 4:(hk + 1) * 4].sum(axis=(0, 1))
+        tot_v = np.abs(dvh[hk]).sum(axis=0)
+        assert np.all(np.abs(dvh[hk].sum(axis=0) - want) <= 2.0 ** -6 * tot_v)

@@ -162,3 +162,13 @@ def test_skipping_a_pair_only_changes_that_tiles_query_gradient():
     changed = np.argwhere(diff > 0)
     assert changed.size and np.all(changed[:, 0] == 0) and np.all(changed[:, 1] == 0)
     assert np.all((changed[:, 2] >= 24) & (changed[:, 2] < 32))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dq_rows_match_the_full_backward(causal):
+    Q, K, V, W, skip, BM, BN = masked_case(31, causal)
+    full = oracle.attention_backward(Q, K, V, W, scale=0.5, causal=causal, skip=skip, BM=BM, BN=BN)
+    rows = [(0, 0, 0), (0, 3, 17), (1, 1, 47), (1, 2, 23), (0, 1, 8)]
+    got = oracle.backward_dq_rows(Q, K, V, W, rows, scale=0.5, causal=causal, skip=skip, BM=BM, BN=BN)
+    want = np.stack([full["dq"][b, h, r] for b, h, r in rows])
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)

@@ -101,3 +101,44 @@ def test_fp8_rejects_wide_tiles_and_bad_scales(bl):
     with pytest.raises(bl.BlasstError) as e:
         bl.decode_fp8(to_dev(inp.q), k8, k8, scale=inp.scale, k_scale=0.0, v_scale=1.0)
     assert e.value.status == 1
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("lam", [0.0, 0.05])
+def test_fp8_full_size_sampled(bl, lam):
+    # the benchmarked FP8 launch: batch 32, Hq 32 / Hkv 8, 32768-key cache, 16 splits, per-tensor
+    # scales; the oracle runs on sampled (sequence, KV head) tiles of the decoded cache
+    inp = planted_decode(32, 32, 8, 32768, 128, seed=3, reading="blk")
+    k, v = to_dev(inp.k), to_dev(inp.v)
+
+    def quant(x):  # on the device: the same nearest-even, saturating cast as synth.e4m3_bits
+        sc = float(x.float().abs().max().item()) / 448.0
+        return (x.float() / sc).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8), sc
+
+    k8, ks = quant(k)
+    v8, vs = quant(v)
+    del k, v
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse, mask, cnt = bl.decode_fp8(to_dev(inp.q), k8, v8, scale=inp.scale, k_scale=ks, v_scale=vs, lam=lam,
+                                      num_splits=16, status_word=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    rng = np.random.default_rng(2)
+    tiles = np.sort(rng.choice(32 * 8, 8, replace=False))
+    kdeq = np.zeros_like(inp.k)
+    vdeq = np.zeros_like(inp.v)
+    for t in tiles:
+        b, h = divmod(int(t), 8)
+        kdeq[b, h] = bf16_bits(e4m3_to_f32(k8[b, h].cpu().numpy()))
+        vdeq[b, h] = bf16_bits(e4m3_to_f32(v8[b, h].cpu().numpy()))
+    bits = unpack_mask(mask.cpu().numpy(), 512)
+    kw = dict(scale=inp.scale * ks, lam=lam, causal=False, is_decode=True, num_splits=16, BN=64, tiles=tiles)
+    ref = oracle.attention(inp.q, kdeq, vdeq, **kw)
+    nd, _ = compare_masks(bits, ref, lam, tiles)
+    assert nd == 0, f"{nd} mask bits differ outside the band"
+    fr = oracle.attention(inp.q, kdeq, vdeq, forced_skip=bits, **kw)
+    sel = np.zeros((32, 32, 1), bool)
+    for t in tiles:
+        b, h = divmod(int(t), 8)
+        sel[b, h * 4:(h + 1) * 4, :] = True
+    assert_outputs_close(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64), fr["o"] * vs, fr["lse"], sel)

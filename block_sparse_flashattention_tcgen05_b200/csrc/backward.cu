@@ -37,10 +37,11 @@
 // dV [256,384); dK [384,512).
 //
 // MMA issue order per pair t: dP(t) [after the dQ^T(t-1) columns are read],
-// then, once dS^T(t) is ready: dQ^T(t), dV(t), S(t+1), dK(t).  The compute
-// warps form P(t+1) from S(t+1) while dK(t) and dP(t+1) run.  Operations
-// issued by one thread execute in issue order, so S(t+1) overwrites P^T(t)
-// only after dV(t) has read it, and a commit covers every earlier operation.
+// then, once dS^T(t) is ready: dQ^T(t), dV(t), S(t+1), dK(t) -- or dK(t)
+// before S(t+1) when pair t+1's Q tile has not landed yet.  The compute warps
+// form P(t+1) from S(t+1) while dK(t) and dP(t+1) run.  Operations issued by
+// one thread execute in issue order, so S(t+1) overwrites P^T(t) only after
+// dV(t) has read it, and a commit covers every earlier operation.
 #include <climits>
 
 #include <cuda_bf16.h>

@@ -187,6 +187,15 @@ def to_pinned(a):
 
 
 # --------------------------------------------------------------------- workloads
+def workload_name(kind, cfg):
+    """The config name both bench arms print for a workload built on a base config."""
+    if kind == "backward":
+        return "fixed-mask backward, " + cfg["workload"]
+    if kind == "decode_fp8":
+        return cfg["workload"] + ", FP8 (e4m3) K/V cache"
+    return cfg["workload"]
+
+
 class Prefill:
     kind = "prefill"
     unit = "TFLOP/s"
@@ -253,6 +262,7 @@ class Backward(Prefill):
             self.__dict__.update({k: v for k, v in fwd.__dict__.items() if k not in ("o", "lse")})
         else:
             super().__init__(cfg, device)
+        self.cfg = dict(self.cfg, workload=workload_name("backward", self.cfg))
         import synth
 
         c = self.cfg
@@ -392,7 +402,7 @@ class DecodeFp8(Decode):
         import torch
 
         self.__dict__.update(src.__dict__)
-        self.cfg = dict(src.cfg, workload=src.cfg["workload"] + ", FP8 (e4m3) K/V cache")
+        self.cfg = dict(src.cfg, workload=workload_name("decode_fp8", src.cfg))
 
         def quant(x):
             sc = float(x.float().abs().max().item()) / 448.0
@@ -899,6 +909,7 @@ def run_reference(args, world, rank):
         return
     wl_kind = args.workload
     cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2, "backward": 0, "decode_fp8": 1}[wl_kind]]
+    cfg = dict(cfg, workload=workload_name(wl_kind, cfg))
     per_step = []
     vals = []
     budget = float(os.environ.get("BLASST_REF_STEP_SECONDS", "8"))

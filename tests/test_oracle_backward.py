@@ -172,3 +172,28 @@ def test_dq_rows_match_the_full_backward(causal):
     got = oracle.backward_dq_rows(Q, K, V, W, rows, scale=0.5, causal=causal, skip=skip, BM=BM, BN=BN)
     want = np.stack([full["dq"][b, h, r] for b, h, r in rows])
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_two_key_closed_form():
+    """One query, two keys (blocks of one key): with p = sigmoid(s0 - s1) the gradient is
+    dq = scale p (1-p) (dO.(v0 - v1)) (k0 - k1), dk0 = -dk1 = scale p (1-p) (dO.(v0 - v1)) q,
+    dv0 = p dO, dv1 = (1 - p) dO; skipping key 1's block leaves dq = dk = 0, dv0 = dO, dv1 = 0."""
+    rng = np.random.default_rng(41)
+    d = 5
+    q = rng.standard_normal((1, 1, 1, d))
+    k = rng.standard_normal((1, 1, 2, d))
+    v = rng.standard_normal((1, 1, 2, d))
+    do = rng.standard_normal((1, 1, 1, d))
+    scale = 0.8
+    s0, s1 = scale * q[0, 0, 0] @ k[0, 0, 0], scale * q[0, 0, 0] @ k[0, 0, 1]
+    p = 1.0 / (1.0 + math.exp(s1 - s0))
+    g = p * (1 - p) * (do[0, 0, 0] @ (v[0, 0, 0] - v[0, 0, 1]))
+    out = oracle.attention_backward(q, k, v, do, scale=scale, causal=False, BM=1, BN=1)
+    np.testing.assert_allclose(out["dq"][0, 0, 0], scale * g * (k[0, 0, 0] - k[0, 0, 1]), atol=1e-13)
+    np.testing.assert_allclose(out["dk"][0, 0, 0], scale * g * q[0, 0, 0], atol=1e-13)
+    np.testing.assert_allclose(out["dk"][0, 0, 1], -scale * g * q[0, 0, 0], atol=1e-13)
+    np.testing.assert_allclose(out["dv"][0, 0], np.stack([p * do[0, 0, 0], (1 - p) * do[0, 0, 0]]), atol=1e-13)
+    skipped = oracle.attention_backward(q, k, v, do, scale=scale, causal=False, BM=1, BN=1,
+                                        skip=np.array([[0, 1]], np.uint8))
+    assert np.all(skipped["dq"] == 0) and np.all(skipped["dk"] == 0)
+    np.testing.assert_allclose(skipped["dv"][0, 0], np.stack([do[0, 0, 0], np.zeros(d)]), atol=1e-15)

@@ -200,3 +200,20 @@ def test_backward_full_size_sampled_rows_and_invariants(bl):
         want = dov[hk * 4:(hk + 1) * 4].sum(axis=(0, 1))
         tot_v = np.abs(dvh[hk]).sum(axis=0)
         assert np.all(np.abs(dvh[hk].sum(axis=0) - want) <= 2.0 ** -6 * tot_v)
+
+
+def test_backward_noncausal_more_queries_than_keys(bl):
+    inp = random_normal(1, 4, 2, 500, 200, 128, seed=68)
+    check_backward(bl, inp, 0.0, False, seed=8)
+
+
+def test_backward_group_of_sixteen(bl):
+    inp = planted_prefill(1, 16, 1, 384, 128, seed=69, reading="blk")
+    check_backward(bl, inp, 0.1, True, seed=9)
+
+
+@pytest.mark.parametrize("lam", [0.5, 0.999])
+def test_backward_heavy_skipping_batch_three_ragged(bl, lam):
+    inp = planted_prefill(3, 2, 1, 250 + 128 * 3, 128, seed=70, reading="blk")
+    _, bits, _ = check_backward(bl, inp, lam, True, seed=10)
+    assert bits.any()

@@ -142,3 +142,10 @@ def test_fp8_full_size_sampled(bl, lam):
         b, h = divmod(int(t), 8)
         sel[b, h * 4:(h + 1) * 4, :] = True
     assert_outputs_close(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64), fr["o"] * vs, fr["lse"], sel)
+
+
+def test_fp8_cache_shorter_than_a_block_more_splits_than_blocks(bl):
+    inp = planted_decode(3, 8, 2, 40, 128, seed=77, reading="blk")
+    check_fp8(bl, inp, 0.05, 4)
+    inp = planted_decode(2, 8, 2, 64 * 3 + 1, 128, seed=78, reading="blk")
+    check_fp8(bl, inp, 0.3, 16)

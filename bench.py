@@ -41,6 +41,8 @@ sys.path.insert(0, ROOT)
 METRIC = "prefill eff. TFLOP/s & decode eff. HBM GB/s at 0/50/75% sparsity (1×B200)"
 FLOP_PER_PAIR = 2 * 128 * 128 * 128
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# spec-sheet figures of one B200, for context beside the measured denominators
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, Hq=32, Hkv=8, L=32768, d=128,
                causal=True, seed=2)
@@ -596,6 +598,75 @@ class Mla:
         return work / (ms * 1e-3) / 1e9
 
 
+def r4(x):
+    """Four significant digits (the JSON line stays short enough to be read whole)."""
+    return None if x is None else float(f"{x:.4g}")
+
+
+def per_head_sparsity(wl, lam):
+    """Skipped / visited pairs of each head at lambda (one extra call with the skip
+    mask, outside any timed region): (min, median, max) over the heads.  Prefill:
+    each query head (its tiles' pairs); decode: each KV head, over the batch (the
+    tile of a decode is a KV head's group)."""
+    import numpy as np
+    import torch
+
+    c = wl.cfg
+    wl.count = torch.zeros(1, dtype=torch.int64, device=wl.device)
+    if wl.kind in ("prefill", "backward"):
+        nq = (c["L"] + 127) // 128
+        nb = (c["L"] + 127) // 128
+        _, _, m, _ = wl.bl.prefill(wl.q, wl.k, wl.v, scale=wl.inp.scale, lam=lam, causal=True, o=wl.o,
+                                   lse=wl.lse, skip_mask=True, skip_count=wl.count)
+        heads, rows_per_head = c["B"] * c["Hq"], nq
+        vis = np.full(c["Hq"], wl.visited / heads)
+    else:
+        nb = (c["Lk"] + 63) // 64
+        _, _, m, _ = wl.bl.decode(wl.q, wl.k, wl.v, scale=wl.inp.scale, lam=lam, num_splits=c["splits"], o=wl.o,
+                                  lse=wl.lse, skip_mask=True, skip_count=wl.count, workspace=wl.ws,
+                                  seed_splits=getattr(wl, "seed_splits", False))
+        heads, rows_per_head = c["Hkv"], 1
+        vis = np.full(c["Hkv"], float(c["B"] * nb))
+    torch.cuda.synchronize()
+    w = m.cpu().numpy().astype(np.uint32)
+    ones = np.zeros(w.shape[0], np.int64)
+    for bit in range(32):
+        ones += ((w >> np.uint32(bit)) & np.uint32(1)).sum(axis=1)
+    if wl.kind in ("prefill", "backward"):
+        per = ones.reshape(c["B"], c["Hq"], rows_per_head).sum(axis=(0, 2)) / vis
+    else:
+        per = ones.reshape(c["B"], c["Hkv"]).sum(axis=0) / vis
+    return [r4(float(per.min())), r4(float(np.median(per))), r4(float(per.max()))]
+
+
+def decision_overhead(wl, flush, rounds=4, per_round=3):
+    """The prefill against its measurement instance with the skip decision compiled
+    out, both at lambda = 0 (the same dense result), timed in interleaved rounds:
+    (median ms of each, speed of the real kernel relative to the no-vote one)."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    t = {"vote": [], "novote": []}
+    fns = {"vote": wl.bl.prefill, "novote": wl.bl.measure_prefill_novote}
+    for name, fn in fns.items():  # warm-up
+        for _ in range(2):
+            fn(wl.q, wl.k, wl.v, scale=wl.inp.scale, lam=0.0, causal=True, o=wl.o, lse=wl.lse, skip_mask=False,
+               skip_count=False)
+    for _ in range(rounds):
+        for name, fn in fns.items():
+            for _ in range(per_round):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                flush.zero_()
+                a.record(stream)
+                fn(wl.q, wl.k, wl.v, scale=wl.inp.scale, lam=0.0, causal=True, o=wl.o, lse=wl.lse,
+                   skip_mask=False, skip_count=False)
+                b.record(stream)
+                torch.cuda.synchronize()
+                t[name].append(a.elapsed_time(b))
+    mv, mn = statistics.median(t["vote"]), statistics.median(t["novote"])
+    return {"ms": r4(mv), "ms_no_vote": r4(mn), "speed_vs_no_vote": r4(mn / mv), "pages": "0.96-1.00"}
+
+
 def lambdas_for_targets(wl, gaps):
     out = {}
     for t in TARGETS:
@@ -953,8 +1024,12 @@ def main():
     ap.add_argument("--no-mqa", action="store_true", help="skip the 128-head MQA decode rows of the sweep")
     ap.add_argument("--no-backward", action="store_true", help="skip the fixed-mask backward rows of the sweep")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-cache decode rows of the sweep")
-    ap.add_argument("--calibration", action="store_true",
-                    help="also fit lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K} (64K GQA prefill shape)")
+    ap.add_argument("--no-calibration", action="store_true",
+                    help="skip the fit of lambda*L = alpha*exp(beta*s) over L in {8K,16K,32K,64K}")
+    ap.add_argument("--no-decision-overhead", action="store_true",
+                    help="skip timing the prefill against its no-vote instance at lambda = 0")
+    ap.add_argument("--detail-out", default=None,
+                    help="also write every sweep point in full (lambda, a = lambda*L, ...) to this JSON file")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -1040,7 +1115,7 @@ def main():
         roof["ncu_source"] = prof.get("source")
 
     # ---- sweep: 0/50/75% on every workload, speedup over lambda = 0
-    sweep = {}
+    sweep, sweep_full = {}, {}
     if not args.no_sweep:
         if "prefill" not in wls:
             try:
@@ -1077,7 +1152,6 @@ def main():
                 lams[k] = w.lambdas() if hasattr(w, "lambdas") else lambdas_for_targets(w, w.calibrate())
         rounds = 4
         for kind, w in wls.items():
-            rows = {}
             # the sparsity points of a workload are timed round-robin, so that a drift of
             # clocks or temperature during the sweep lands on all of them alike
             times = {t: [] for t in TARGETS}
@@ -1088,30 +1162,52 @@ def main():
                                                       3 if rnd == 0 else 1, flush)
                     times[t] += ms_t
             base = statistics.median(times[0.0])
+            pk = peaks["bf16_tflops"] if w.bound == "tensor" else peaks["hbm_gbs"]
+            spk = SPEC_PEAKS["bf16_tflops"] if w.bound == "tensor" else SPEC_PEAKS["hbm_gbs"]
+            pts, full = [], {}
             for t in TARGETS:
                 lam = lams[kind][t][0]
                 sk = sk_by_t[t]
                 med = statistics.median(times[t])
                 r = w.rate(w.work(sk), med)
-                pk = peaks["bf16_tflops"] if w.bound == "tensor" else peaks["hbm_gbs"]
-                rows[f"{int(t * 100)}%"] = {
-                    "lambda": lam, "a=lambda*L": lam * (w.cfg.get("L") or w.cfg.get("Lk")),
-                    "sparsity": sk / w.visited, "ms": med, "value": r, "unit": w.unit,
-                    "frac_of_measured_peak": r / pk, "speedup_vs_lambda0": base / med}
-                if w.kind == "prefill":
-                    # each skipped pair omits its 128 x 128 exponentials: the skipped-exp share is the sparsity
-                    rows[f"{int(t * 100)}%"]["exp_skipped_fraction"] = sk / w.visited
-                if hasattr(w, "flops"):
+                pt = [r4(sk / w.visited), r4(med), r4(r), r4(r / pk), r4(r / spk), r4(base / med)]
+                row = {"lambda": lam, "a=lambda*L": lam * (w.cfg.get("L") or w.cfg.get("Lk")),
+                       "sparsity": sk / w.visited, "ms": med, "value": r, "unit": w.unit,
+                       "frac_of_measured_peak": r / pk, "frac_of_spec_peak": r / spk, "speedup_vs_lambda0": base / med}
+                if hasattr(w, "flops"):  # MLA: the tensor side too
                     tf = w.flops(sk) / (med * 1e-3) / 1e12
-                    rows[f"{int(t * 100)}%"].update(tflops=tf, tensor_frac_of_measured_peak=tf / peaks["bf16_tflops"])
-            rows["max_reachable_sparsity"] = lams[kind]["max"][1]
-            sweep[kind] = rows
+                    pt.append(r4(tf / peaks["bf16_tflops"]))
+                    row.update(tflops=tf, tensor_frac_of_measured_peak=tf / peaks["bf16_tflops"])
+                pts.append(pt)
+                full[f"{int(t * 100)}%"] = row
+            full["max_reachable_sparsity"] = lams[kind]["max"][1]
+            sweep[kind] = {"u": w.unit, "pts": pts, "max_s": r4(lams[kind]["max"][1])}
+            sweep_full[kind] = full
+
+    # ---- per-head sparsity distribution at the ~75% point (A10: report the per-head distribution)
+    per_head = {}
+    for kind in ("prefill", "prefill_64k", "decode"):
+        if kind in wls and kind in lams:
+            per_head[kind] = per_head_sparsity(wls[kind], lams[kind][0.75][0])
+
+    # ---- the decision's cost: prefill against its no-vote instance at lambda = 0
+    dec_ovh = None
+    if not args.no_decision_overhead and "prefill" in wls:
+        dec_ovh = decision_overhead(wls["prefill"], flush)
 
     # ---- calibration fit across context lengths (prefill-shaped decision pass)
-    calib = None
-    if args.calibration and "prefill" in wls:
+    calib = calib_full = None
+    if not args.no_calibration and "prefill" in wls:
         lengths = (8192, 16384, 32768, 65536) if args.size == "full" else (2048, 4096, 8192)
-        calib = calibration_sweep(dev, lengths)
+        calib_full = calibration_sweep(dev, lengths)
+        err_by_L = {}
+        for row in calib_full["per_point"]:
+            err_by_L.setdefault(str(row["L"]), []).append(row["abs_error"])
+        calib = {"alpha": r4(calib_full["alpha"]), "beta": r4(calib_full["beta"]), "points": calib_full["points"],
+                 "mean_abs_err": r4(calib_full["mean_abs_sparsity_error"]),
+                 "max_abs_err": r4(calib_full["max_abs_sparsity_error"]),
+                 "mean_abs_err_by_L": {L: r4(statistics.mean(v)) for L, v in err_by_L.items()},
+                 "targets": [0.3, 0.4, 0.5, 0.6, 0.7, 0.8]}
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -1136,13 +1232,26 @@ def main():
     for k in ("B", "Hq", "Hkv", "L", "Lk", "d", "splits"):
         if k in wl.cfg:
             cfgd[k] = wl.cfg[k]
+    roof["frac_of_spec"] = roof["achieved"] / (SPEC_PEAKS["bf16_tflops"] if wl.bound == "tensor"
+                                              else SPEC_PEAKS["hbm_gbs"])
+    roof["spec_peak"] = SPEC_PEAKS["bf16_tflops"] if wl.bound == "tensor" else SPEC_PEAKS["hbm_gbs"]
     line = {
         "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfgd,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": wl.launches * args.steps,
-        "clocks": clocks, "sweep": sweep, "calibration": calib, "notes": notes,
+        "clocks": clocks, "notes": notes,
+        # the keys below are kept short and last, so that a reader of the line's tail sees all of them
+        "decision_overhead": dec_ovh, "per_head_sparsity_75": per_head, "calibration": calib,
+        "sweep_cols": ["sparsity", "ms", "value", "frac_measured", "frac_spec", "speedup_vs_lambda0",
+                       "(mla) tensor_frac_measured"],
+        "sweep": sweep,
     }
+    if args.detail_out and rank == 0:
+        with open(args.detail_out, "w") as f:
+            json.dump({"line": line, "sweep": sweep_full, "calibration": calib_full,
+                       "lambdas": {k: {str(t): v for t, v in d.items()} for k, d in lams.items()}}, f, indent=1,
+                      default=str)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -73,7 +73,8 @@ def lib() -> ctypes.CDLL:
             raise ImportError(f"{LIB_PATH} is missing: build it with "
                               "`python -m block_sparse_flashattention_tcgen05_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
-        for name in ("blasst_prefill", "blasst_decode", "blasst_calibrate", "blasst_decode_noalloc"):
+        for name in ("blasst_prefill", "blasst_decode", "blasst_calibrate", "blasst_decode_noalloc",
+                     "blasst_measure_prefill_novote"):
             f = getattr(L, name)
             f.restype = ctypes.c_int
             f.argtypes = _ATTN_ARGS
@@ -162,7 +163,7 @@ def _attn(fn_name, q, k, v, *, scale, lam, causal, o, lse, want_mask, want_count
 
 
 def prefill(q, k, v, *, scale, lam=0.0, causal=True, o=None, lse=None, skip_mask=True, skip_count=True,
-            status_word=None, stream=None):
+            status_word=None, stream=None, _entry="blasst_prefill"):
     """Prefill attention with block skipping.  q [B,Hq,Lq,128], k/v [B,Hkv,Lk,128] bf16 on CUDA.
 
     Returns (o, lse, skip_mask [B*Hq*ceil(Lq/128), W] int32 or None, skip_count [1] int64 or None).
@@ -179,10 +180,17 @@ def prefill(q, k, v, *, scale, lam=0.0, causal=True, o=None, lse=None, skip_mask
     opts = Opts(status_word=None if status_word is None else status_word.data_ptr())
     nq = (Lq + 127) // 128
     nb = (Lk + 127) // 128
-    m, c = _attn("blasst_prefill", q, k, v, scale=scale, lam=lam, causal=causal, o=o, lse=lse,
+    m, c = _attn(_entry, q, k, v, scale=scale, lam=lam, causal=causal, o=o, lse=lse,
                  want_mask=skip_mask, want_count=skip_count, opts=opts, stream=stream, mask_rows=B * Hq * nq,
                  n_blocks=nb, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=d)
     return o, lse, m, c
+
+
+def measure_prefill_novote(q, k, v, **kw):
+    """blasst_measure_prefill_novote (include/blasst_measure.h): prefill() with
+    the skip decision compiled out, every visited block kept.  Measurement only:
+    timed against prefill() at lam = 0 it gives the decision's cost."""
+    return prefill(q, k, v, _entry="blasst_measure_prefill_novote", **kw)
 
 
 def prefill_backward(q, k, v, o, lse, dout, *, scale, causal=True, skip_mask=None, dq=None, dk=None, dv=None,
@@ -299,8 +307,8 @@ def decode_fp8(q, k8, v8, *, scale, k_scale, v_scale, lam=0.0, causal=False, num
     return o, lse, mask, count
 
 
-def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=None, lse=None, skip_mask=True,
-                   skip_count=True, status_word=None, stream=None):
+def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=None, dv=None, o=None, lse=None,
+                   skip_mask=True, skip_count=True, status_word=None, stream=None):
     """Same as decode(), through blasst_decode_noalloc: the library allocates
     nothing (split partials in its fixed device array).  Output tensors that
     are not passed are created here, by the caller side of the interface."""
@@ -308,13 +316,14 @@ def decode_noalloc(q, k, v, *, scale, lam=0.0, causal=False, num_splits=16, o=No
 
     _dev_tensor(q, "q"), _dev_tensor(k, "k"), _dev_tensor(v, "v")
     B, Hq, Lq, d = q.shape
-    _, Hkv, Lk, _ = k.shape
-    dv = v.shape[-1]
+    _, Hkv, Lk, krs = k.shape
+    vrs = v.shape[-1]
+    dv = vrs if dv is None else dv
     if o is None:
         o = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    opts = Opts(num_splits=num_splits, dv=dv,
+    opts = Opts(num_splits=num_splits or 0, dv=dv, k_row_stride=krs, v_row_stride=vrs,
                 status_word=None if status_word is None else status_word.data_ptr())
     nb = (Lk + 63) // 64
     m, c = _attn("blasst_decode_noalloc", q, k, v, scale=scale, lam=lam, causal=causal, o=o, lse=lse,

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/blasst.h"
+#include "../../include/blasst_measure.h"
 #include "internal.h"
 
 using namespace blasst;
@@ -134,6 +135,30 @@ float log2_threshold(float lambda) {
 
 const double kLog2e = 1.4426950408889634;
 
+}  // namespace
+
+blasst_status blasst::decode_split_count(int d, int num_splits, int B, int Hkv, int Lk, int *out) {
+    *out = 0;
+    if (num_splits > 0) {
+        *out = num_splits;
+        return BLASST_OK;
+    }
+    if (num_splits == 0) {
+        *out = d == 576 ? 2 : 16;  // MLA: two CTAs per split already fill the device at batch 64
+        return BLASST_OK;
+    }
+    if (num_splits != -1 || d == 576) return BLASST_ERR_INVALID;
+    // adaptive: from the batch, the cache length and this device's SM count
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(multiprocessors)");
+    *out = blasst_decode_pick_splits(B, Hkv, Lk, sms);
+    return BLASST_OK;
+}
+
+namespace {
+
 // ---------------------------------------------------------------------- MLA
 blasst_status run_mla(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                       int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
@@ -144,8 +169,10 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
     if (!calib && (v != k || c.vrs != c.krs)) return BLASST_ERR_UNSUPPORTED;
     const long long R = (long long)Hq * Lq;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
-    const int S = op.num_splits ? op.num_splits : 2;
-    if (S < 1 || S > 65535 || B > 65535) return BLASST_ERR_INVALID;
+    int S = 0;
+    blasst_status sst = decode_split_count(d, op.num_splits, B, Hkv, Lk, &S);
+    if (sst != BLASST_OK) return sst;
+    if (S > 65535 || B > 65535) return BLASST_ERR_INVALID;
     const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
     const int per_split = (nb + S - 1) / S;
     const int words = (nb + 31) / 32;
@@ -256,15 +283,10 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     const bool wide = R > 16;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
     if (wide && op.seed_splits) return BLASST_ERR_UNSUPPORTED;
-    int S = op.num_splits ? op.num_splits : 16;
-    if (S == -1) {  // adaptive: from the batch, the cache length and this device's SM count
-        int dev = 0, sms = 0;
-        cudaError_t ed = cudaGetDevice(&dev);
-        if (ed == cudaSuccess) ed = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (ed != cudaSuccess) return cuda_fail(ed, "cudaDeviceGetAttribute(multiprocessors)");
-        S = blasst_decode_pick_splits(B, Hkv, Lk, sms);
-    }
-    if (S < 1 || S > 65535) return BLASST_ERR_INVALID;
+    int S = 0;
+    st = decode_split_count(d, op.num_splits, B, Hkv, Lk, &S);
+    if (st != BLASST_OK) return st;
+    if (S > 65535) return BLASST_ERR_INVALID;
     if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + S - 1) / S > 1024)
         return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 blocks per split
     if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;
@@ -373,7 +395,8 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
 // ------------------------------------------------------------------ prefill
 blasst_status run_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
                           int Lq, int Lk, int d, float scale, float lambda, int causal, uint32_t *skip_mask,
-                          unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib) {
+                          unsigned long long *skip_count, void *stream, const blasst_opts *opts_in, bool calib,
+                          bool novote = false) {
     blasst_opts op = read_opts(opts_in);
     Common c;
     blasst_status st = check_common(q, k, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, op, &c);
@@ -422,7 +445,7 @@ blasst_status run_prefill(const void *q, const void *k, const void *v, void *o, 
     p.causal = causal ? 1 : 0;
     p.scale_log2 = (float)(scale * kLog2e);
     p.thr_log2 = log2_threshold(lambda);
-    e = launch_prefill(p, tq, tk, tv, calib, sm);
+    e = novote ? launch_prefill_novote(p, tq, tk, tv, sm) : launch_prefill(p, tq, tk, tv, calib, sm);
     if (e == cudaErrorNotSupported) return BLASST_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return cuda_fail(e, "prefill kernel");
     return BLASST_OK;
@@ -527,6 +550,14 @@ blasst_status blasst_prefill(const void *q, const void *k, const void *v, void *
                              unsigned long long *skip_count, void *stream, const blasst_opts *opts) {
     return run_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
                        opts, false);
+}
+
+blasst_status blasst_measure_prefill_novote(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                                            int Hq, int Hkv, int Lq, int Lk, int d, float scale, float lambda,
+                                            int causal, uint32_t *skip_mask, unsigned long long *skip_count,
+                                            void *stream, const blasst_opts *opts) {
+    return run_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, lambda, causal, skip_mask, skip_count, stream,
+                       opts, false, true);
 }
 
 blasst_status blasst_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,

@@ -30,33 +30,63 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchB
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+// One resolved address per (device, context).  A context made current through the
+// driver API is a different context from the runtime's primary one, and the array
+// has a different address in each.
+struct ScratchAddr {
+    int dev;
+    CUcontext ctx;
+    void *addr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
+int g_n_scratch_addr = 0;
 
-// Device address of the scratch array on the current device; resolved once
-// per device (the first call on a device loads the module there).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    }
+    return fn;
+}
+
+blasst_status fail(const char *what, cudaError_t e) {
+    char msg[160];
+    std::snprintf(msg, sizeof msg, "%s: %s", what, cudaGetErrorString(e));
+    blasst::set_last_error(msg);
+    return BLASST_ERR_CUDA;
+}
+
+// Device address of the scratch array for the current device and context.  The
+// first call there resolves it (cudaGetSymbolAddress, which loads this module on
+// the device); later calls reuse the cached address.
 blasst_status scratch_for_current_device(void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        char msg[160];
-        std::snprintf(msg, sizeof msg, "cudaGetDevice: %s",
-                      e == cudaSuccess ? "device index out of range" : cudaGetErrorString(e));
-        blasst::set_last_error(msg);
-        return BLASST_ERR_CUDA;
-    }
+    if (e != cudaSuccess) return fail("cudaGetDevice", e);
+    CUcontext ctx = nullptr;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx) get_ctx(&ctx);  // null before the runtime has made a context current
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess || !p) {
-            char msg[160];
-            std::snprintf(msg, sizeof msg, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-            blasst::set_last_error(msg);
-            return BLASST_ERR_CUDA;
+    for (int i = 0; i < g_n_scratch_addr; i++) {
+        if (g_scratch_addr[i].dev == dev && g_scratch_addr[i].ctx == ctx && ctx) {
+            *out = g_scratch_addr[i].addr;
+            return BLASST_OK;
         }
-        g_scratch_addr[dev] = p;
     }
-    *out = g_scratch_addr[dev];
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || !p) return fail("cudaGetSymbolAddress(scratch)", e);
+    if (!ctx && get_ctx) get_ctx(&ctx);  // the lookup above made the primary context current
+    if (ctx && g_n_scratch_addr < kMaxDevices) g_scratch_addr[g_n_scratch_addr++] = ScratchAddr{dev, ctx, p};
+    *out = p;
     return BLASST_OK;
 }
 
@@ -74,9 +104,15 @@ BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, con
     if (opts) std::memcpy(&op, opts, opts->struct_size < sizeof op ? opts->struct_size : sizeof op);
     op.struct_size = sizeof op;
     if (op.workspace) return BLASST_ERR_INVALID;  // the scratch is the library's, not the caller's
-    const int splits = op.num_splits ? op.num_splits : 16;
-    if (B <= 0 || Hq <= 0 || Lq <= 0 || splits <= 0) return BLASST_ERR_INVALID;
-    const size_t need = blasst_decode_workspace_bytes(B, Hq, Lq, op.dv, splits);
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return BLASST_ERR_INVALID;
+    // the split count and value width exactly as blasst_decode will resolve them
+    // (MLA defaults to 2 splits, GQA/MQA to 16, -1 to the adaptive count)
+    int splits = 0;
+    blasst_status st = blasst::decode_split_count(d, op.num_splits, B, Hkv, Lk, &splits);
+    if (st != BLASST_OK) return st;
+    op.num_splits = splits;
+    const int dv = op.dv ? op.dv : d;
+    const size_t need = blasst_decode_workspace_bytes(B, Hq, Lq, dv, splits);
     if (need == 0 || need > kNoAllocScratchBytes) {
         char msg[160];
         std::snprintf(msg, sizeof msg, "decode partials need %zu bytes; the fixed scratch holds %zu", need,
@@ -85,7 +121,7 @@ BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, con
         return BLASST_ERR_WORKSPACE;
     }
     void *scratch = nullptr;
-    blasst_status st = scratch_for_current_device(&scratch);
+    st = scratch_for_current_device(&scratch);
     if (st != BLASST_OK) return st;
     // every byte the kernels read from the scratch is written earlier in the
     // same call (each split writes all its partial rows), so nothing is cleared

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/blasst.h"
+
 namespace blasst {
 
 constexpr int kDecodeBlockN = 64;
@@ -98,6 +100,10 @@ cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &tmap_q, const
                             const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, cudaStream_t stream);
 // Records the text returned by blasst_last_error() for this thread.
 void set_last_error(const char *msg);
+// The split count a decode call with these arguments uses: num_splits when positive;
+// 0 -> 16 (d = 128) or 2 (MLA, d = 576); -1 -> blasst_decode_pick_splits with the current
+// device's SM count (d = 128 only; BLASST_ERR_INVALID for MLA and other negative values).
+blasst_status decode_split_count(int d, int num_splits, int B, int Hkv, int Lk, int *out);
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
                           int nt, cudaStream_t stream);
@@ -112,5 +118,8 @@ cudaError_t launch_mla(const MlaParams &p, const CUtensorMap &tmap_q, const CUte
                        cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
                            const CUtensorMap &tmap_v, bool calib, cudaStream_t stream);
+// The prefill with the skip decision compiled out (measurement instance; never used by the API).
+cudaError_t launch_prefill_novote(const PrefillParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                                  const CUtensorMap &tmap_v, cudaStream_t stream);
 
 }  // namespace blasst

@@ -20,7 +20,9 @@
 //   MMA:      S_t = Q_t K_j^T           (always, for every visited block)
 //   softmax:  row max m~ of scale*S, true running max M <- max(M, m~),
 //             vote (m~ - M < log2 lambda, or the row sees no key of the
-//             block); bar.red.and over the 128 rows = the tile decision.
+//             block); the tile decision is the AND over the 128 rows, taken
+//             in two levels: __all_sync per warp, then a named barrier that
+//             only warps voting "skip" wait on (the others arrive and go on).
 //             The first block is never skipped.
 //   kept:     lazy rescale of O when the exp reference lags M by > 2^8,
 //             P = 2^(s - M_ref) -> bf16 in TMEM, l += sum P, then
@@ -83,10 +85,15 @@ __device__ __forceinline__ int last_block(const PrefillParams &p, int q0) {
     return min(p.nb - 1, (last_row + p.Lk - p.Lq) >> 7);
 }
 
-template <bool CALIB>
+// MODE 0: attention; 1: decision-only calibration pass; 2: attention with the
+// skip decision compiled out (every visited block kept, no vote, no barrier), a
+// measurement instance that gives the cost of the decision at lambda = 0.
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
+    constexpr bool CALIB = MODE == 1;
+    constexpr bool NOVOTE = MODE == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sq = smem;                                  // Q_A, Q_B
@@ -231,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const bool kept = !CALIB && tl->dec[t] != 0;
+                    const bool kept = NOVOTE || (!CALIB && tl->dec[t] != 0);
                     if (kept) {
                         if (!v_waited) {
                             if (!mbar_wait(&tl->v_full[st], (j / kStagesV) & 1, &tl->abort)) {
@@ -339,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // j, so a barrier instance is complete before its id is used again; the ids
             // also alternate with the block parity.)
             bool skip = false;
-            if (j > 0) {
+            if (!NOVOTE && j > 0) {
                 const bool wvote = __all_sync(0xffffffffu, vote);
                 uint8_t *vb = reinterpret_cast<uint8_t *>(&tl->votes[t][j & 1]);
                 if (lane == 0) vb[wq] = wvote ? 1 : 0;
@@ -363,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 bar_sync(bar_id, kSoftmaxThreads);
             }
-            if (row == 0) tl->dec[t] = skip ? 0 : 1;
+            if (!NOVOTE && row == 0) tl->dec[t] = skip ? 0 : 1;
             if (skip || CALIB) {
                 if (!skip) m_true = mn;
                 __syncwarp();
@@ -487,11 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
-template <bool CALIB>
+template <int MODE>
 cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                      cudaStream_t st) {
-    constexpr int smem = prefill_smem_bytes<CALIB>();
-    auto kern = prefill_kernel<CALIB>;
+    constexpr int smem = prefill_smem_bytes<MODE == 1>();
+    auto kern = prefill_kernel<MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int n_pairs = (p.n_qtiles + 1) / 2;
@@ -504,7 +511,12 @@ cudaError_t launch_t(const PrefillParams &p, const CUtensorMap &tq, const CUtens
 
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                            const CUtensorMap &tv, bool calib, cudaStream_t st) {
-    return calib ? launch_t<true>(p, tq, tk, tv, st) : launch_t<false>(p, tq, tk, tv, st);
+    return calib ? launch_t<1>(p, tq, tk, tv, st) : launch_t<0>(p, tq, tk, tv, st);
+}
+
+cudaError_t launch_prefill_novote(const PrefillParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                  const CUtensorMap &tv, cudaStream_t st) {
+    return launch_t<2>(p, tq, tk, tv, st);
 }
 
 }  // namespace blasst

@@ -82,10 +82,10 @@ typedef struct blasst_opts {
     size_t struct_size;
     int dv;                    /* value head dim; 0 -> d.  MLA: d = 576, dv = 512 */
     int block_n;               /* 0, or the fixed block size (128 prefill, 64 decode) */
-    int num_splits;            /* decode: KV chunks per sequence; 0 -> 16; -1 -> adaptive
-                                  (blasst_decode, _decode_paged, _decode_fp8 with d = 128:
-                                  blasst_decode_pick_splits with this device's SM count;
-                                  MLA and the no-allocation call reject it) */
+    int num_splits;            /* decode: KV chunks per sequence; 0 -> 16 (d = 128) or 2
+                                  (MLA, d = 576); -1 -> adaptive for d = 128
+                                  (blasst_decode_pick_splits with this device's SM count;
+                                  MLA rejects it with BLASST_ERR_INVALID) */
     int mode;                  /* blasst_calibrate only: 0 = prefill tiling, 1 = decode tiling */
     long long k_row_stride;    /* elements between consecutive keys; 0 -> d */
     long long v_row_stride;    /* elements between consecutive values; 0 -> dv */
@@ -271,15 +271,19 @@ BLASST_API blasst_status blasst_calibrate_threshold(const float *gaps, long long
  *   - calls needing more than BLASST_NOALLOC_SCRATCH_BYTES of partials
  *     (blasst_decode_workspace_bytes) return BLASST_ERR_WORKSPACE with the
  *     sizes in blasst_last_error();
- *   - the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, which loads the module on that device); make
- *     that first call before any stream capture;
+ *   - the first call on each device (in each CUDA context) looks up the
+ *     array's device address (cudaGetSymbolAddress, which loads the module
+ *     on that device) and caches it for later calls in that context; make
+ *     that first call before any stream capture.  The cached address does
+ *     not survive cudaDeviceReset: after a reset of a device, do not call
+ *     this function on that device again in the same process;
  *   - every call on a device shares the one array and it keeps the last
  *     call's contents (nothing in it needs clearing: each call writes every
  *     partial it reads), so calls that may overlap on the GPU -- on different
  *     streams or from different host threads -- race: serialise them.
- * It calls no cudaMalloc, cudaMallocAsync, cudaFree or other allocating
- * routine.
+ * num_splits (0, positive or -1) and dv are resolved exactly as blasst_decode
+ * resolves them before the size check.  It calls no cudaMalloc,
+ * cudaMallocAsync, cudaFree or other allocating routine.
  */
 #define BLASST_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -28,9 +28,12 @@ def bl():
 
 
 def declared_symbols():
-    with open(os.path.join(ROOT, "include", "blasst.h")) as f:
-        text = f.read()
-    return re.findall(r"BLASST_API\s+[\w\s\*]+?\b(blasst_\w+)\s*\(", text)
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            with open(os.path.join(ROOT, "include", h)) as f:
+                names += re.findall(r"BLASST_API\s+[\w\s\*]+?\b(blasst_\w+)\s*\(", f.read())
+    return names
 
 
 def test_exports_every_declared_symbol(bl):
@@ -186,8 +189,25 @@ def test_pick_splits(bl):
 def test_adaptive_splits_only_where_supported(bl):
     mla = dict(num_splits=-1, dv=512, k_row_stride=576, v_row_stride=576)
     assert _call(bl, "blasst_decode", d=576, opts=bl.Opts(**mla)) == 1   # MLA
-    assert _call(bl, "blasst_decode_noalloc", opts=bl.Opts(num_splits=-1)) == 1
+    assert _call(bl, "blasst_decode_noalloc", d=576, opts=bl.Opts(**mla)) == 1
     assert _call(bl, "blasst_decode", opts=bl.Opts(num_splits=-2)) == 1
+    assert _call(bl, "blasst_decode_noalloc", opts=bl.Opts(num_splits=-2)) == 1
+
+
+def test_noalloc_sizes_partials_as_the_decode_does(bl):
+    """The no-allocation call sizes its partials with the split count and value
+    width blasst_decode will use: MLA (d = 576, dv = 512) defaults to 2 splits,
+    so batch 4 x 128 heads needs about 2 MiB and passes the size check, while
+    16 splits at batch 64 exceed the fixed array and are refused up front."""
+    mla = dict(dv=512, k_row_stride=576, v_row_stride=576)
+    limit = bl.NOALLOC_SCRATCH_BYTES
+    assert bl.decode_workspace_bytes(4, 128, 1, 512, 2) < limit < bl.decode_workspace_bytes(4, 128, 1, 512, 16)
+    # the 2-split size passes; what follows needs the device (no device here: a CUDA error, not a size error)
+    assert _call(bl, "blasst_decode_noalloc", B=4, Hq=128, d=576, opts=bl.Opts(**mla)) != 3
+    assert bl.decode_workspace_bytes(64, 128, 1, 512, 16) > limit
+    assert _call(bl, "blasst_decode_noalloc", B=64, Hq=128, d=576, opts=bl.Opts(num_splits=16, **mla)) == 3
+    assert _call(bl, "blasst_decode_noalloc", B=64, Hq=128, opts=bl.Opts(num_splits=16)) == 3
+    assert _call(bl, "blasst_decode_noalloc", opts=bl.Opts(workspace=FAKE, workspace_bytes=1 << 20)) == 1
 
 
 def test_calibrate_requires_gaps_and_valid_mode(bl):

@@ -194,3 +194,16 @@ def test_prefill_64k_sampled(bl):
     nq = 512
     tiles = [nq - 1, 5 * nq + 200, 17 * nq + 3, 31 * nq + nq - 1]
     check_prefill(bl, inp, 3e-3, True, tiles=tiles)
+
+
+def test_prefill_novote_instance_equals_dense_prefill(bl):
+    # the measurement instance (decision compiled out) computes, at lambda = 0,
+    # exactly what the real kernel computes there: nothing is skipped by either
+    inp = planted_prefill(1, 4, 2, 1000, 128, seed=8, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    o1, l1, m1, c1 = bl.prefill(q, k, v, scale=inp.scale, lam=0.0, causal=True)
+    o2, l2, m2, c2 = bl.measure_prefill_novote(q, k, v, scale=inp.scale, lam=0.0, causal=True)
+    torch.cuda.synchronize()
+    assert int(c1.item()) == 0 and int(c2.item()) == 0
+    assert torch.equal(m1, m2) and torch.equal(o1, o2) and torch.equal(l1, l2)
+    check_prefill(bl, inp, 0.0, True)

@@ -631,7 +631,7 @@ def per_head_sparsity(wl, lam):
     w = m.cpu().numpy().astype(np.uint32)
     ones = np.zeros(w.shape[0], np.int64)
     for bit in range(32):
-        ones += ((w >> np.uint32(bit)) & np.uint32(1)).sum(axis=1)
+        ones += ((w >> np.uint32(bit)) & np.uint32(1)).astype(np.int64).sum(axis=1)
     if wl.kind in ("prefill", "backward"):
         per = ones.reshape(c["B"], c["Hq"], rows_per_head).sum(axis=(0, 2)) / vis
     else:

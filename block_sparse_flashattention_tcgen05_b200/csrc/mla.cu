@@ -572,48 +572,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         unsigned int n_skip = 0;
         uint32_t mword = 0;
         int mword_idx = -1;
+        // An own block's scores come out of tensor memory, and its row maxima go to the
+        // partner, one block AHEAD of its decision: while waiting for the maxima of the
+        // partner's block in front of it.  The two CTAs therefore never wait on each
+        // other's decisions to send their own maxima.
+        float s[64];    // scores of the next own block (log2 units after scaling in the exp)
+        float mt_own = NEG_INF;
+        int n_read = 0;  // own blocks read so far
+        auto read_own = [&](int jo) {  // S of own block jo -> s[], row max -> partner
+            const int o = jo >> 1;
+            if (!mbar_wait(&tl->s_full, o & 1, &tl->abort)) set_timeout(tl, p.status);
+            tc_fence_after();
+            {
+                uint32_t *sr = reinterpret_cast<uint32_t *>(s);
+                tmem_ld32(s_addr, sr);
+                tmem_ld32(s_addr + 32, sr + 32);
+                tc_wait_ld();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->s_free);  // the next own S may overwrite it now
+            const int lim = last_key - (j0 + jo) * kBN;
+            if (lim < kBN - 1) {
+#pragma unroll
+                for (int c = 0; c < kBN; c++)
+                    if (c > lim) s[c] = NEG_INF;
+            }
+            float m0 = NEG_INF, m1 = NEG_INF, m2 = NEG_INF, m3 = NEG_INF;
+#pragma unroll
+            for (int c = 0; c < kBN; c += 8) {
+                m0 = fmax3(m0, s[c], s[c + 1]);
+                m1 = fmax3(m1, s[c + 2], s[c + 3]);
+                m2 = fmax3(m2, s[c + 4], s[c + 5]);
+                m3 = fmax3(m3, s[c + 6], s[c + 7]);
+            }
+            mt_own = fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
+            const int slot = o % kMx;
+            if (o >= kMx && !mbar_wait_cluster(&tl->mx_empty[slot], ((o / kMx) - 1) & 1, &tl->abort))
+                set_timeout(tl, p.status);
+            st_cluster_f32(peer_mx_in + (uint32_t)(slot * kRows * 4), mt_own);
+            fence_acq_rel_cluster();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(peer_mx_full + (uint32_t)(slot * 8));
+            n_read++;
+        };
         for (int jj = 0; jj < nblk; jj++) {
             const int j = j0 + jj;
             const bool own = (uint32_t)(jj & 1) == h;
             const int o = jj >> 1;  // index among the owner's blocks
-            float s[64];
             float mt;
             if (own) {
-                if (!mbar_wait(&tl->s_full, o & 1, &tl->abort)) set_timeout(tl, p.status);
-                tc_fence_after();
-                {
-                    uint32_t *sr = reinterpret_cast<uint32_t *>(s);
-                    tmem_ld32(s_addr, sr);
-                    tmem_ld32(s_addr + 32, sr + 32);
-                    tc_wait_ld();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tl->s_free);
-                const int lim = last_key - j * kBN;
-                if (lim < kBN - 1) {
-#pragma unroll
-                    for (int c = 0; c < kBN; c++)
-                        if (c > lim) s[c] = NEG_INF;
-                }
-                float m0 = NEG_INF, m1 = NEG_INF, m2 = NEG_INF, m3 = NEG_INF;
-#pragma unroll
-                for (int c = 0; c < kBN; c += 8) {
-                    m0 = fmax3(m0, s[c], s[c + 1]);
-                    m1 = fmax3(m1, s[c + 2], s[c + 3]);
-                    m2 = fmax3(m2, s[c + 4], s[c + 5]);
-                    m3 = fmax3(m3, s[c + 6], s[c + 7]);
-                }
-                mt = fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
-                // hand the row maxima to the partner
-                const int slot = o % kMx;
-                if (o >= kMx && !mbar_wait_cluster(&tl->mx_empty[slot], ((o / kMx) - 1) & 1, &tl->abort))
-                    set_timeout(tl, p.status);
-                st_cluster_f32(peer_mx_in + (uint32_t)(slot * kRows * 4), mt);
-                fence_acq_rel_cluster();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(peer_mx_full + (uint32_t)(slot * 8));
+                if (n_read <= o) read_own(jj);  // (only the first own block of CTA 0 is read here)
+                mt = mt_own;
             } else {
+                if (jj + 1 < nblk) read_own(jj + 1);  // the next block is ours: read and send it first
                 const int slot = o % kMx;
                 if (!mbar_wait_cluster(&tl->mx_full[slot], (o / kMx) & 1, &tl->abort)) set_timeout(tl, p.status);
                 mt = tl->mx_in[slot][row];

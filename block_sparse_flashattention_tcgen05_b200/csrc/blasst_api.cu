@@ -216,6 +216,7 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
     p.causal = causal ? 1 : 0;
     p.scale_log2 = (float)(scale * kLog2e);
     p.thr_log2 = log2_threshold(lambda);
+    p.seed = op.seed_splits ? 1 : 0;
     e = launch_mla(p, tq, tk, calib, sm);
     if (e != cudaSuccess) return cuda_fail(e, "MLA split kernel");
     if (!calib) {
@@ -266,7 +267,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         return BLASST_ERR_INVALID;
     }
     if (op.block_n != 0 && op.block_n != kDecodeBlockN) return BLASST_ERR_UNSUPPORTED;
-    if (op.seed_splits && d != 128) return BLASST_ERR_UNSUPPORTED;  // split seeding: GQA/MQA decode only
+    if (op.seed_splits && d != 128 && d != 576) return BLASST_ERR_UNSUPPORTED;  // split seeding: decode only
     if (pg && (d != 128 || c.dv != 128 || c.krs != d || c.vrs != c.dv)) return BLASST_ERR_UNSUPPORTED;
     if (f8) {
         if (!(std::isfinite(f8->k_scale) && f8->k_scale > 0.f && std::isfinite(f8->v_scale) && f8->v_scale > 0.f))

@@ -93,6 +93,7 @@ struct MlaParams {
     int causal;
     float scale_log2;
     float thr_log2;
+    int seed;                       // 1: splits after the first start from block 0's row maxima
 };
 
 // prep (delta, lse2, zeroed dQ accumulator), the main tcgen05 kernel, dq finalize

@@ -96,7 +96,8 @@ typedef struct blasst_opts {
                                   tile's (split's) first block, NaN if not visited */
     unsigned int *status_word; /* device word the caller zeroes; the library ORs in
                                   a nonzero code when a bounded wait expires */
-    int seed_splits;           /* decode (d = 128) only: nonzero seeds the running
+    int seed_splits;           /* decode only (d = 128 tiles of up to 16 rows, and MLA):
+                                  nonzero seeds the running
                                   max of every split after the first with the row
                                   maxima of block 0, and such a split has no forced
                                   first block.  Block 0 enters those splits only

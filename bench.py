@@ -47,8 +47,8 @@ SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, Hq=32, Hkv=8, L=32768, d=128,
                causal=True, seed=2)
 DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk=32768, d=128, splits=16, seed=3)
-MLA = dict(workload="MLA decode, 128 heads, 576/512 latent, 32K cache, 2 splits", B=64, Hq=128, Lk=32768, splits=2,
-           seed=5)
+MLA = dict(workload="MLA decode, 128 heads, 576/512 latent, 32K cache, 8 seeded splits", B=64, Hq=128, Lk=32768,
+           splits=8, seed_splits=True, seed=5)
 MQA = dict(workload="decode MQA, 128 query heads on one KV head, 32K cache, 16 splits", B=64, Hq=128, Hkv=1,
            Lk=32768, d=128, splits=16, seed=9)
 PREFILL_64K = dict(PREFILL, workload="prefill GQA 64K (Qwen3-8B-like attention shape)", L=65536, seed=4)
@@ -567,13 +567,14 @@ class Mla:
 
     def calibrate(self):
         gaps, _, _ = self.bl.calibrate(self.q, self.k, scale=self.inp.scale, causal=False, mode="decode",
-                                       num_splits=self.cfg["splits"], dv=512)
+                                       num_splits=self.cfg["splits"], dv=512,
+                                       seed_splits=self.cfg.get("seed_splits", False))
         return gaps.cpu().numpy()
 
     def call(self, lam, stream=None):
         return self.bl.decode(self.q, self.k, self.k, scale=self.inp.scale, lam=lam, num_splits=self.cfg["splits"],
                               dv=512, o=self.o, lse=self.lse, skip_mask=False, skip_count=self.count,
-                              workspace=self.ws, stream=stream)
+                              workspace=self.ws, stream=stream, seed_splits=self.cfg.get("seed_splits", False))
 
     def work(self, skipped):
         c = self.cfg
@@ -820,7 +821,7 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
         cand = list(range(inp.q.shape[0]))
         rng.shuffle(cand)
         kw = dict(scale=inp.scale, causal=False, is_decode=True, num_splits=c["splits"], BN=64, dv=512,
-                  v_row_stride=576)
+                  v_row_stride=576, seed_splits=c.get("seed_splits", False))
         n_tiles = c["B"]
 
         def units(r):

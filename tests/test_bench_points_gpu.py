@@ -193,7 +193,7 @@ def test_decode_fp8_at_bench_lambda(dev, target):
     assert int(cnt.item()) == int(bits.sum())
 
 
-@pytest.mark.parametrize("target", (0.5, 0.75))
+@pytest.mark.parametrize("target", TARGETS)
 def test_mla_at_bench_lambda(dev, target):
     import block_sparse_flashattention_tcgen05_b200 as bl
 
@@ -203,8 +203,9 @@ def test_mla_at_bench_lambda(dev, target):
     B, Hq, Lq, _ = inp.q.shape
     splits = wl.cfg["splits"]
     st = torch.zeros(1, dtype=torch.int32, device=dev)
+    seeded = wl.cfg.get("seed_splits", False)
     o, lse, mask, cnt = bl.decode(wl.q, wl.k, wl.k, scale=inp.scale, lam=lam, num_splits=splits, dv=512,
-                                  status_word=st)
+                                  status_word=st, seed_splits=seeded)
     torch.cuda.synchronize()
     assert st.item() == 0
     assert abs(int(cnt.item()) / wl.visited - achieved) < 1e-9, "sparsity differs from the calibration's"
@@ -212,7 +213,7 @@ def test_mla_at_bench_lambda(dev, target):
     bits = unpack_mask(mask.cpu().numpy(), nb)
     tiles = [0, B // 2 + int(target * 10), B - 1]
     kw = dict(scale=inp.scale, lam=lam, causal=False, is_decode=True, num_splits=splits, BN=64, dv=512,
-              v_row_stride=576, tiles=tiles)
+              v_row_stride=576, tiles=tiles, seed_splits=seeded)
     ref = oracle.attention(inp.q, inp.k, inp.k, **kw)
     nd, _ = compare_masks(bits, ref, lam, tiles)
     assert nd == 0, f"{nd} mask bits differ outside the band"

@@ -50,8 +50,7 @@ struct DecodeSmemTail {
     uint64_t k_empty[8];
     uint64_t v_full[8];
     uint64_t v_empty[8];
-    uint64_t red_full[4];  // block row maxima of all consumer warps published (one arrival per warp)
-    float red[4][kConsumerWarps][16];
+    float red[2][kConsumerWarps][16];
     float lred[kConsumerWarps][16];
     float rred[kConsumerWarps][16];
     float mfin[16];
@@ -112,7 +111,7 @@ __device__ __forceinline__ int2 kv_block_coord(const DecodeParams &p, int b, int
 }
 
 template <int NT, int NK, int NV, bool CALIB, bool F8>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
     decode_split_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v) {
     extern __shared__ uint8_t smem_raw[];
@@ -177,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
                 mbar_init(&tl->v_empty[i], kConsumerWarps);
             }
         }
-        for (int i = 0; i < 4; i++) mbar_init(&tl->red_full[i], kConsumerWarps);
         tl->dec_count = 0;
         tl->abort = 0;
         fence_mbar_init();
@@ -437,10 +435,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         if (nent > 0) convert_k(0);
     }
 
-    // Scores of ring entry e: S^T = K_e q^T for my 16 keys, scaled and masked (log2 units), and
-    // my warp's per-column maxima published in red[e % 4] (one arrival on red_full[e % 4]).
-    auto score = [&](int e, float (&s)[NT][4]) {
-        const int jj = e - seed;
+    for (int e = 0; e < nent; e++) {
+        const int jj = e - seed;  // block index within the split; -1: the seed block
         const int j = jj < 0 ? 0 : j0 + jj;
         const int slot = e % NK;
         if (!F8 && !mbar_wait(&tl->k_full[slot], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
@@ -478,62 +474,43 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 
         // scaled, masked scores in log2 units; my keys: lo = g4, hi = g4 + 8
         const int key_lo = j * kDecodeBlockN + warp * 16 + g4;
+        float s[NT][4];
         float cmax[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) {
 #pragma unroll
-            for (int u = 0; u < 2; u++) {
-                s[nt][u] = key_lo <= lastk[nt][u] && key_lo < Lk ? acc[nt][u] * p.scale_log2 : NEG_INF;
-                s[nt][2 + u] = key_lo + 8 <= lastk[nt][u] && key_lo + 8 < Lk ? acc[nt][2 + u] * p.scale_log2 : NEG_INF;
-                float m = fmaxf(s[nt][u], s[nt][2 + u]);
+            for (int e = 0; e < 2; e++) {
+                s[nt][e] = key_lo <= lastk[nt][e] && key_lo < Lk ? acc[nt][e] * p.scale_log2 : NEG_INF;
+                s[nt][2 + e] = key_lo + 8 <= lastk[nt][e] && key_lo + 8 < Lk ? acc[nt][2 + e] * p.scale_log2 : NEG_INF;
+                float m = fmaxf(s[nt][e], s[nt][2 + e]);
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-                cmax[nt][u] = m;
+                cmax[nt][e] = m;
             }
         }
-        // red[e % 4] was last read for entry e - 4; every warp finished that read before it
-        // published entry e - 2, which this warp has waited for
         if (g4 == 0) {
 #pragma unroll
             for (int nt = 0; nt < NT; nt++) {
-                tl->red[e & 3][warp][nt * 8 + 2 * t4] = cmax[nt][0];
-                tl->red[e & 3][warp][nt * 8 + 2 * t4 + 1] = cmax[nt][1];
+                tl->red[e & 1][warp][nt * 8 + 2 * t4] = cmax[nt][0];
+                tl->red[e & 1][warp][nt * 8 + 2 * t4 + 1] = cmax[nt][1];
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tl->red_full[e & 3]);
-    };
-
-    // Software pipeline over the ring entries: entry e+1 is scored and published before
-    // the warps wait for each other's maxima of entry e, so that the wait overlaps
-    // the next block's tensor-core work instead of following it.
-    float s[NT][4];
-    if (nent > 0) score(0, s);
-    for (int e = 0; e < nent; e++) {
-        const int jj = e - seed;  // block index within the split; -1: the seed block
-        const int j = jj < 0 ? 0 : j0 + jj;
-        float s_next[NT][4];
-        if (e + 1 < nent) {
-            if constexpr (F8) convert_k(e + 1);
-            score(e + 1, s_next);
+        if constexpr (F8) {
+            if (e + 1 < nent) convert_k(e + 1);  // overlaps the other warps reaching the barrier
         }
-        if (!mbar_wait(&tl->red_full[e & 3], (e >> 2) & 1, &tl->abort)) set_timeout(tl, p.status);
+        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 
         if (jj < 0) {
             // the seed block: its row maxima start the running max of this split
 #pragma unroll
             for (int c = 0; c < NC; c++) {
-                float mt = tl->red[e & 3][0][c];
+                float mt = tl->red[e & 1][0][c];
 #pragma unroll
-                for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 3][w][c]);
+                for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 1][w][c]);
                 Mall[c] = mt;
             }
             seen = true;  // no forced first block after a seed
-#pragma unroll
-            for (int nt = 0; nt < NT; nt++)
-#pragma unroll
-                for (int i = 0; i < 4; i++) s[nt][i] = s_next[nt][i];
             continue;
         }
 
@@ -543,9 +520,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         bool visited = false;
 #pragma unroll
         for (int c = 0; c < NC; c++) {
-            float mt = tl->red[e & 3][0][c];
+            float mt = tl->red[e & 1][0][c];
 #pragma unroll
-            for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 3][w][c]);
+            for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 1][w][c]);
             Mn[c] = fmaxf(Mall[c], mt);
             if (mt > NEG_INF) {
                 visited = true;
@@ -610,10 +587,6 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
         }
         push_pop(kept, cs, cmo, cmn);
         }
-#pragma unroll
-        for (int nt = 0; nt < NT; nt++)
-#pragma unroll
-            for (int i = 0; i < 4; i++) s[nt][i] = s_next[nt][i];
     }
     if constexpr (!CALIB) {
         // the last queued blocks

@@ -15,7 +15,11 @@
 // producer of Q (once) and K (2-stage ring), warp 5 TMEM allocation + tcgen05.mma
 // issue, warp 6 V producer (2-stage ring, kept blocks only).  Two CTAs share an SM
 // (99 KB of shared memory and 256 TMEM columns each).
-// TMEM (256 columns): S [0,64), P [64,96) bf16, O [128,256).
+// TMEM (256 columns): S [0,64), P [64,128) as two bf16 buffers, O [128,256).
+// A K stage goes back to its producer as soon as S has read it, and kept blocks
+// alternate between the two P buffers, so the softmax writes P(k) once the P.V of
+// kept block k-2 (not k-1) is done: two V loads stay in flight behind the
+// decisions instead of one.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -34,15 +38,17 @@ constexpr int kStageBytes = 2 * kBoxBytesKV;
 constexpr int kQBytes = 2 * kBoxBytesQ;
 constexpr int kNK = 2, kNV = 2;   // two CTAs per SM: each keeps two blocks of K and of V in flight
 constexpr int kMaxWideBlocks = 1024;  // blocks per split (decision array)
-constexpr uint32_t kColP = 64, kColO = 128;
+constexpr uint32_t kColP = 64, kColO = 128;  // P buffer b at kColP + 32 b
+constexpr int kDecRing = 8;                    // decisions published ahead of the MMA thread
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusBadPage = 2;
 
 struct WideSmemTail {
     uint64_t q_full, k_full[kNK], k_empty[kNK], v_full[kNV], v_empty[kNV];
-    uint64_t s_full, s_free, o_done, mma_done;
-    uint64_t p_full[2];  // [block parity]: published at most one block ahead of the MMA warp
+    uint64_t s_full, s_free, mma_done;
+    uint64_t o_done[2];  // [P buffer]: the P.V that read it has completed
+    uint64_t p_full[kDecRing], dec_free[kDecRing];  // block decisions (and P) ready / taken
     uint32_t tmem_base;
     int dec_count;       // decisions published (blocks of this split)
     int abort;
@@ -111,10 +117,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         mbar_init(&tl->s_full, 1);
         mbar_init(&tl->s_free, 4);
-        mbar_init(&tl->o_done, 1);
+        mbar_init(&tl->o_done[0], 1);
+        mbar_init(&tl->o_done[1], 1);
         mbar_init(&tl->mma_done, 1);
-        mbar_init(&tl->p_full[0], 4);
-        mbar_init(&tl->p_full[1], 4);
+        for (int i = 0; i < kDecRing; i++) {
+            mbar_init(&tl->p_full[i], 4);
+            mbar_init(&tl->dec_free[i], 1);
+        }
         tl->dec_count = 0;
         tl->abort = 0;
         fence_mbar_init();
@@ -206,9 +215,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     umma_ss2(s_col, q_lo + qo, kst + ko, dhi, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&tl->s_full);
+                umma_commit(&tl->k_empty[jj % kNK]);  // K is read by S only
             };
             // S(ns) once the softmax holds S(ns-1) in registers and K(ns) landed; block
-            // np's decision as it arrives (P.V when kept, then K stage and V stage back)
+            // np's decision as it arrives (P.V when kept, then its V stage back)
             int n_pv = 0, ns = 0, np = 0, vk = 0;
             long long t_last = clock64();
             while (ok && np < nblk) {
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     ns++;
                     did = true;
                 }
-                if (np < ns && mbar_test_wait(&tl->p_full[np & 1], (np >> 1) & 1)) {
+                if (np < ns && mbar_test_wait(&tl->p_full[np % kDecRing], (np / kDecRing) & 1)) {
                     tc_fence_after();
                     if (!CALIB && dec[np]) {
                         const int st = vk % kNV;
@@ -231,16 +241,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                         }
                         tc_fence_after();
                         const uint32_t vst = v_lo + (uint32_t)((st * kStageBytes) >> 4);
+                        const uint32_t pb = p_col + (uint32_t)((n_pv & 1) * 32);
 #pragma unroll
                         for (int kk = 0; kk < kBN / 16; kk++)
-                            umma_ts2(o_col, p_col + kk * 8, vst + (uint32_t)((kk * 16 * 128) >> 4), dhi, idesc_pv,
+                            umma_ts2(o_col, pb + kk * 8, vst + (uint32_t)((kk * 16 * 128) >> 4), dhi, idesc_pv,
                                      (n_pv > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit(&tl->o_done);
+                        umma_commit(&tl->o_done[n_pv & 1]);
                         umma_commit(&tl->v_empty[st]);
                         n_pv++;
                         vk++;
                     }
-                    umma_commit(&tl->k_empty[np % kNK]);
+                    mbar_arrive(&tl->dec_free[np % kDecRing]);
                     np++;
                     did = true;
                 }
@@ -272,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         int mword_idx = -1;
         for (int jj = 0; jj < nblk; jj++) {
             const int j = j0 + jj;
-            const int sl = jj & 1;
+            const int sl = jj % kDecRing;
             if (!mbar_wait(&tl->s_full, jj & 1, &tl->abort)) set_timeout(tl, p.status);
             tc_fence_after();
             float s[64];
@@ -309,6 +320,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             seen = seen || visited;
             const bool skip = visited && all && !first;
             const bool kept = visited && !skip;
+            // the MMA thread has taken the decision published kDecRing blocks ago
+            if (jj >= kDecRing && !mbar_wait(&tl->dec_free[sl], ((jj / kDecRing) - 1) & 1, &tl->abort))
+                set_timeout(tl, p.status);
             if (row == 0) {
                 // the V producer reads the decision before this block's exponentials run
                 dec[jj] = kept ? 1 : 0;
@@ -343,12 +357,18 @@ __global__ void __launch_bounds__(kThreads, 2)
                     if (mn != NEG_INF) m_ref = mn;
                 }
                 const float mref = m_ref == NEG_INF ? 0.f : m_ref;
-                // P has one buffer: the previous P.V has to have read it
-                if (n_kept > 0) {
-                    if (!mbar_wait(&tl->o_done, (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
+                // P buffer n_kept & 1 was last read by the P.V of kept block n_kept - 2;
+                // rescaling O needs every earlier P.V done (they complete in issue order)
+                const int pbuf = n_kept & 1;
+                if (warp_need && n_kept > 0) {
+                    if (!mbar_wait(&tl->o_done[(n_kept - 1) & 1], ((n_kept - 1) >> 1) & 1, &tl->abort))
+                        set_timeout(tl, p.status);
+                    tc_fence_after();
+                } else if (n_kept >= 2) {
+                    if (!mbar_wait(&tl->o_done[pbuf], ((n_kept - 2) >> 1) & 1, &tl->abort)) set_timeout(tl, p.status);
                     tc_fence_after();
                 }
-                const uint32_t p_addr = tmem + lane_off + kColP;
+                const uint32_t p_addr = tmem + lane_off + kColP + (uint32_t)(pbuf * 32);
                 float rs = 0.f, rr = 0.f;
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
@@ -400,7 +420,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             // split epilogue: normalised partial O and the split's lse for each valid row
             const size_t orow = ((size_t)(b * p.Hq + hkv * p.G) * p.Lq + row) * p.num_splits + split;
             if (n_kept > 0) {
-                if (!mbar_wait(&tl->o_done, (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
+                if (!mbar_wait(&tl->o_done[(n_kept - 1) & 1], ((n_kept - 1) >> 1) & 1, &tl->abort))
+                    set_timeout(tl, p.status);
                 tc_fence_after();
             }
             const float inv = lr > 0.f ? 1.f / lr : 0.f;

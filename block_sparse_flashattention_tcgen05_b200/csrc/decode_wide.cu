@@ -230,16 +230,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     ns++;
                     did = true;
                 }
-                if (np < ns && mbar_test_wait(&tl->p_full[np % kDecRing], (np / kDecRing) & 1)) {
+                // (a kept block whose V has not landed yet waits here without holding up S)
+                if (np < ns && mbar_test_wait(&tl->p_full[np % kDecRing], (np / kDecRing) & 1) &&
+                    (CALIB || !dec[np] || mbar_test_wait(&tl->v_full[vk % kNV], (vk / kNV) & 1))) {
                     tc_fence_after();
                     if (!CALIB && dec[np]) {
                         const int st = vk % kNV;
-                        if (!mbar_wait(&tl->v_full[st], (vk / kNV) & 1, &tl->abort)) {
-                            set_timeout(tl, p.status);
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
                         const uint32_t vst = v_lo + (uint32_t)((st * kStageBytes) >> 4);
                         const uint32_t pb = p_col + (uint32_t)((n_pv & 1) * 32);
 #pragma unroll
@@ -315,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float mn = fmaxf(m_true, mt);
             const bool vote = (mt == NEG_INF) || (mt - mn < p.thr_log2);
             const bool all = bar_and(1, 128, vote);
-            const bool visited = !bar_and(1, 128, mt == NEG_INF);
+            // Every block of the split below the sequence's length is visited: row Lq-1 of
+            // the first head sees keys up to Lk - 1 (bottom-right alignment).
+            const bool visited = true;
             const bool first = visited && !seen;
             seen = seen || visited;
             const bool skip = visited && all && !first;

@@ -64,6 +64,11 @@ SIZES = {"full": (PREFILL, DECODE, MLA), "medium": (MEDIUM_PREFILL, MEDIUM_DECOD
 TARGETS = (0.0, 0.5, 0.75)
 
 
+def mqa_cfg(size, dcfg):
+    """The 128-head MQA decode at the benchmark size, or a smaller batch at the other sizes."""
+    return MQA if size == "full" else dict(MQA, B=max(2, MQA["B"] // 8), Lk=dcfg["Lk"])
+
+
 # --------------------------------------------------------------------------- utils
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -980,7 +985,10 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     wl_kind = args.workload
-    cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2, "backward": 0, "decode_fp8": 1}[wl_kind]]
+    if wl_kind == "decode_mqa":
+        cfg = mqa_cfg(args.size, SIZES[args.size][1])
+    else:
+        cfg = SIZES[args.size][{"prefill": 0, "decode": 1, "mla": 2, "backward": 0, "decode_fp8": 1}[wl_kind]]
     cfg = dict(cfg, workload=workload_name(wl_kind, cfg))
     per_step = []
     vals = []
@@ -1012,7 +1020,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--workload", choices=["prefill", "decode", "mla", "backward", "decode_fp8"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "decode", "mla", "backward", "decode_fp8", "decode_mqa"],
+                    default="prefill")
     ap.add_argument("--size", choices=sorted(SIZES), default="full",
                     help="full = the benchmark shapes; medium = profiling size; quick = smoke-testing the bench")
     ap.add_argument("--no-sweep", action="store_true")
@@ -1073,6 +1082,8 @@ def main():
         wls["decode_fp8"] = DecodeFp8(wls["decode"], dev)
     if headline_kind == "mla":
         wls["mla"] = Mla(mcfg, dev)
+    if headline_kind == "decode_mqa":
+        wls["decode_mqa"] = DecodeMqa(mqa_cfg(args.size, dcfg), dev)
     if headline_kind == "backward":
         wls["backward"] = Backward(pcfg, dev)
         wls["backward"].count = torch.zeros(1, dtype=torch.int64, device=dev)
@@ -1135,9 +1146,8 @@ def main():
         if not args.no_paged:
             wls["decode_paged"] = DecodePaged(wls["decode"], dev,
                                               min_len=min(8192, wls["decode"].cfg["Lk"] // 4))
-        if not args.no_mqa:
-            mcfg_q = MQA if args.size == "full" else dict(MQA, B=max(2, MQA["B"] // 8), Lk=dcfg["Lk"])
-            wls["decode_mqa"] = DecodeMqa(mcfg_q, dev)
+        if not args.no_mqa and "decode_mqa" not in wls:
+            wls["decode_mqa"] = DecodeMqa(mqa_cfg(args.size, dcfg), dev)
         if "mla" not in wls and not args.no_mla:
             wls["mla"] = Mla(mcfg, dev)
         if "prefill" in wls and "backward" not in wls and not args.no_backward:

@@ -256,3 +256,53 @@ def test_decode_paged_at_bench_lambda(dev, target):
         assert nd == 0, f"sequence {b}: {nd} mask bits differ outside the band"
         fr = oracle.attention(qb, kb, vb, forced_skip=bits[b, :, :nbk], **kw)
         assert_outputs_close(og[b:b + 1], lg[b:b + 1], fr["o"], fr["lse"])
+
+
+@pytest.mark.parametrize("target", TARGETS)
+def test_backward_at_bench_lambda(dev, target):
+    """The fixed-mask backward the bench times: the 32K GQA prefill inputs, the forward's mask at the
+    bench's lambda, the bench's upstream gradient.  Sampled dq rows against the oracle's row function
+    within the per-element bound of tests/test_backward_gpu.py (bf16 dS, the bf16 forward O in D, the
+    output rounding), and over every key sum_k dK_k = 0 and sum_k dV_k = the group's sum of dO rows."""
+    import block_sparse_flashattention_tcgen05_b200 as bl
+    from synth import upstream_grad
+
+    wl, lams = workload("prefill", dev)
+    lam, achieved = lams[target]
+    inp = wl.inp
+    B, Hq, L, _ = inp.q.shape
+    Hkv = inp.k.shape[1]
+    G = Hq // Hkv
+    o, lse, mask, cnt = bl.prefill(wl.q, wl.k, wl.v, scale=inp.scale, lam=lam, causal=True)
+    do_bits = upstream_grad(B, Hq, L, 128, seed=wl.cfg["seed"])  # the bench's dO (bench.Backward)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    dq, dk, dv = bl.prefill_backward(wl.q, wl.k, wl.v, o, lse, bench.to_dev(do_bits, dev), scale=inp.scale,
+                                     causal=True, skip_mask=mask, status_word=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert abs(int(cnt.item()) / wl.visited - achieved) < 1e-9
+    bits = unpack_mask(mask.cpu().numpy(), (L + 127) // 128)
+    rows = [(0, 0, 0), (0, 3, 4097), (0, 9, 12345), (0, 17, 20000), (0, 26, 30001), (0, Hq - 1, L - 1)]
+    ref = oracle.backward_dq_rows(inp.q, inp.k, inp.v, do_bits, rows, scale=inp.scale, causal=True, skip=bits,
+                                  terms=True)
+    dqh = dq.float().cpu().numpy()
+    Kf = bf16_to_f32(inp.k).astype(np.float64)[0]
+    Vf = bf16_to_f32(inp.v).astype(np.float64)[0]
+    Dof = bf16_to_f32(do_bits).astype(np.float64)[0]
+    for n, (b, h, r) in enumerate(rows):
+        kk, vv = Kf[h // G], Vf[h // G]
+        p_, ds_, o_ = ref["P"][n], ref["dS"][n], ref["O"][n]
+        dD = (np.abs(Dof[h, r]) * (2.0 ** -8 * (p_ @ np.abs(vv)) + 2.0 ** -9 * np.abs(o_))).sum()
+        bound = (2.0 ** -9 * (np.abs(ref["dq"][n]) + inp.scale * (np.abs(ds_) @ np.abs(kk))) +
+                 inp.scale * dD * (p_ @ np.abs(kk)))
+        err = np.abs(dqh[b, h, r] - ref["dq"][n])
+        assert np.all(err <= bound + 1e-7), f"row {(b, h, r)}: worst {np.max(err / (bound + 1e-7)):.2f} of bound"
+    dkh = dk.double().cpu().numpy()[0]
+    dvh = dv.double().cpu().numpy()[0]
+    dov = torch.from_numpy(do_bits.view(np.int16)).view(torch.bfloat16).double().numpy()[0]
+    for hk in range(Hkv):
+        tot = np.abs(dkh[hk]).sum(axis=0)
+        assert np.all(np.abs(dkh[hk].sum(axis=0)) <= 2.0 ** -6 * tot)
+        want = dov[hk * G:(hk + 1) * G].sum(axis=(0, 1))
+        tot_v = np.abs(dvh[hk]).sum(axis=0)
+        assert np.all(np.abs(dvh[hk].sum(axis=0) - want) <= 2.0 ** -6 * tot_v)

@@ -15,13 +15,15 @@
 // removes any exchange of scores between SMs.
 //
 // Q (128 x 576 bf16) is split between tensor memory and shared memory: 64-column
-// boxes 0..4 live in TMEM (A operand of tcgen05.mma from TMEM), boxes 5..8 in
+// boxes 0..3 live in TMEM (A operand of tcgen05.mma from TMEM), boxes 4..8 in
 // shared memory.  That leaves a 2-stage ring of whole K blocks (9 boxes, 72 KB).
 //
 // Warp roles (192 threads per CTA): warps 0-3 softmax/decision (thread = row),
-// warp 4 TMA producer (Q boxes 5..8 once, each K block), warp 5 TMEM allocation
+// warp 4 TMA producer (Q boxes 4..8 once, each K block), warp 5 TMEM allocation
 // + tcgen05.mma issue.
-// TMEM: S [0,64), P [64,96) (bf16), Q boxes 0..4 [96,256) (bf16), O_half [256,512).
+// TMEM: S [0,64), P [64,128) (two bf16 buffers: kept blocks alternate, so the
+// softmax writes P(k) once the P.V of kept block k-2 is done), Q boxes 0..3
+// [128,256) (bf16), O_half [256,512).
 //
 // Per block: S (always), tile decision as in the other kernels (true running
 // max, restarted per split, first visited block kept); kept blocks: lazy O
@@ -41,19 +43,20 @@ constexpr int kThreads = 192;
 constexpr int kRows = 128;
 constexpr int kBN = 64;
 constexpr int kBoxes = 9;                       // 576 = 9 x 64 contraction columns
-constexpr int kQTmemBoxes = 5;                  // Q boxes 0..4 in TMEM, 5..8 in shared memory
+constexpr int kQTmemBoxes = 4;                  // Q boxes 0..3 in TMEM, 4..8 in shared memory
 constexpr int kQBoxBytes = kRows * 128;         // 128 rows x 64 bf16
 constexpr int kKBoxBytes = kBN * 128;           // 64 keys x 64 bf16
 constexpr int kStages = 2;
 constexpr int kKStageBytes = kBoxes * kKBoxBytes;                 // 72 KB
-constexpr int kQSmemBytes = (kBoxes - kQTmemBoxes) * kQBoxBytes;  // 64 KB
-constexpr uint32_t kColP = 64, kColQ = 96, kColO = 256;
+constexpr int kQSmemBytes = (kBoxes - kQTmemBoxes) * kQBoxBytes;  // 80 KB
+constexpr uint32_t kColP = 64, kColQ = 128, kColO = 256;  // P buffer b at kColP + 32 b
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kStatusTimeout = 1;
 
 struct MlaSmemTail {
     uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t q_full, qt_full, s_full, s_free, o_done, mma_done;
+    uint64_t q_full, qt_full, s_full, s_free, mma_done;
+    uint64_t o_done[2];  // [P buffer]: the P.V that read it has completed
     // [block parity]: the softmax warps can publish block j+1 before the MMA warp
     // has taken block j, never further ahead
     uint64_t p_full[2];
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmap_k) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sq = smem;                 // Q boxes 5..8
+    uint8_t *sq = smem;                 // Q boxes 4..8
     uint8_t *sk = smem + kQSmemBytes;   // K ring
     MlaSmemTail *tl = reinterpret_cast<MlaSmemTail *>(sk + kStages * kKStageBytes);
 
@@ -101,7 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&tl->qt_full, 4);
         mbar_init(&tl->s_full, 1);
         mbar_init(&tl->s_free, 4);
-        mbar_init(&tl->o_done, 1);
+        mbar_init(&tl->o_done[0], 1);
+        mbar_init(&tl->o_done[1], 1);
         mbar_init(&tl->mma_done, 1);
         mbar_init(&tl->p_full[0], 4);
         mbar_init(&tl->p_full[1], 4);
@@ -200,9 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t vst = v_lo + (uint32_t)(((np % kStages) * kKStageBytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < kBN / 16; kk++)
-                            umma_ts2(o_col, p_col + kk * 8, vst + (uint32_t)((kk * 16 * 128) >> 4), dhi, idesc_pv,
+                            umma_ts2(o_col, p_col + (uint32_t)((n_pv & 1) * 32 + kk * 8),
+                                     vst + (uint32_t)((kk * 16 * 128) >> 4), dhi, idesc_pv,
                                      (n_pv > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit(&tl->o_done);
+                        umma_commit(&tl->o_done[n_pv & 1]);
                         n_pv++;
                     }
                     umma_commit(&tl->k_empty[np % kStages]);
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int last_key = !valid_row ? -1 : (p.causal ? pos + p.Lk - p.Lq : p.Lk - 1);
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const uint32_t s_addr = tmem + lane_off, o_addr = tmem + lane_off + kColO;
-        // Q boxes 0..4 of this row -> TMEM, packed bf16 pairs
+        // Q boxes 0..3 of this row -> TMEM, packed bf16 pairs
         {
             const uint16_t *qrow = p.q + ((size_t)b * p.R + (valid_row ? row : 0)) * 576;
 #pragma unroll 1
@@ -333,12 +338,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mn != NEG_INF) m_ref = mn;
                 }
                 const float mref = m_ref == NEG_INF ? 0.f : m_ref;
-                // P has one buffer: the previous P.V has to have read it
-                if (n_kept > 0) {
-                    if (!mbar_wait(&tl->o_done, (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
+                // Kept blocks alternate between two P buffers: buffer n_kept & 1 was last read by
+                // the P.V of kept block n_kept - 2.  Rescaling O needs every earlier P.V done
+                // (they complete in issue order).
+                const int pbuf = n_kept & 1;
+                if (warp_need && n_kept > 0) {
+                    if (!mbar_wait(&tl->o_done[(n_kept - 1) & 1], ((n_kept - 1) >> 1) & 1, &tl->abort))
+                        set_timeout(tl, p.status);
+                    tc_fence_after();
+                } else if (n_kept >= 2) {
+                    if (!mbar_wait(&tl->o_done[pbuf], ((n_kept - 2) >> 1) & 1, &tl->abort)) set_timeout(tl, p.status);
                     tc_fence_after();
                 }
-                const uint32_t p_addr = tmem + lane_off + kColP;
+                const uint32_t p_addr = tmem + lane_off + kColP + (uint32_t)(pbuf * 32);
                 float rs = 0.f, rr = 0.f;
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
@@ -390,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // split epilogue: normalised partial O (this CTA's 256 value columns), the split's lse
             const size_t orow = ((size_t)b * p.R + row) * p.num_splits + split;
             if (n_kept > 0) {
-                if (!mbar_wait(&tl->o_done, (n_kept - 1) & 1, &tl->abort)) set_timeout(tl, p.status);
+                if (!mbar_wait(&tl->o_done[(n_kept - 1) & 1], ((n_kept - 1) >> 1) & 1, &tl->abort))
+                    set_timeout(tl, p.status);
                 tc_fence_after();
             }
             const float inv = lr > 0.f ? 1.f / lr : 0.f;

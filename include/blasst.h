@@ -142,7 +142,9 @@ BLASST_API blasst_status blasst_decode(const void *q, const void *k, const void 
 /*
  * Decode over an FP8 (e4m3, OCP "E4M3FN": bias 7, no infinities) KV cache.
  * Not on the pages: a storage format that halves the bytes of K and V, which
- * decode reads from HBM once per step.  The cache holds K = k_scale * k8 and
+ * decode reads from HBM once per step.  Experimental: on B200 this kernel is
+ * bound by the conversion of the bytes to f16, not by HBM, and runs slower
+ * than blasst_decode over a bf16 cache; what it saves is the cache's memory.  The cache holds K = k_scale * k8 and
  * V = v_scale * v8 (per-tensor scales, finite and > 0); the arithmetic is
  * exactly blasst_decode's on those dequantized values (same tile, 64-key
  * blocks, splits, skip rule, combine), with one difference in rounding: the

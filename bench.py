@@ -207,6 +207,10 @@ class Prefill:
     kind = "prefill"
     unit = "TFLOP/s"
     bound = "tensor"
+    # end to end: device tensors filled from the host each step, read back each step, and private to a call
+    e2e_in = ("q", "k", "v")
+    e2e_out = ("o", "lse")
+    e2e_private = ()
 
     def __init__(self, cfg, device):
         import synth
@@ -261,6 +265,7 @@ class Backward(Prefill):
     alone (prep, main kernel, dq finalize).  Work: the five 128x128x128 products
     of every kept pair (S, dP, dQ, dV, dK)."""
     kind = "backward"
+    e2e_in = None  # its own end-to-end step (inputs include the forward's o, lse and mask)
 
     def __init__(self, cfg, device, fwd=None):
         import torch
@@ -333,6 +338,9 @@ class Decode:
     unit = "GB/s"
     bound = "hbm"
     seed_splits = False
+    e2e_in = ("q", "k", "v")
+    e2e_out = ("o", "lse")
+    e2e_private = ("ws",)
 
     def __init__(self, cfg, device):
         import synth
@@ -404,6 +412,7 @@ class DecodeFp8(Decode):
     calibration (the sweep reports the sparsity each λ reaches here)."""
 
     kind = "decode_fp8"
+    e2e_in = None  # its own end-to-end step (the e4m3 cache)
 
     def __init__(self, src, device):
         import torch
@@ -548,6 +557,9 @@ class Mla:
     kind = "mla"
     unit = "GB/s"
     bound = "hbm"
+    e2e_in = ("q", "k")  # v is the same tensor as k
+    e2e_out = ("o", "lse")
+    e2e_private = ("ws",)
 
     def __init__(self, cfg, device):
         import synth
@@ -713,6 +725,73 @@ def timed_launches(wl, lam, steps, warmup, flush, sampler=None):
 
 
 def e2e_measure(wl, lam, steps, warmup):
+    """The metric end to end through the public API, from and to pinned host memory.
+
+    Every step copies its inputs host -> device, makes the call and copies its result
+    device -> host, all inside the timed region.  Where the workload names its device
+    tensors (e2e_in / e2e_out), steps run as a pipeline over two sets of device buffers
+    and three streams: step i's host -> device copy overlaps step i-1's call and step
+    i-2's device -> host copy (PCIe carries both directions at once).  Otherwise the
+    workload's own step runs serially on one stream."""
+    import copy
+
+    import torch
+
+    if getattr(wl, "e2e_in", None) is None:
+        return _e2e_serial(wl, lam, steps, warmup)
+    wl.count = torch.zeros(1, dtype=torch.int64, device=wl.device)
+    sets = [wl, copy.copy(wl)]
+    for name in wl.e2e_in + wl.e2e_out + wl.e2e_private + ("count",):
+        setattr(sets[1], name, getattr(wl, name).clone())
+    if isinstance(wl, Mla):
+        sets[1].v = sets[1].k
+    host_in = {name: getattr(wl, name).cpu().pin_memory() for name in wl.e2e_in}
+    host_out = [{name: torch.empty(getattr(wl, name).shape, dtype=getattr(wl, name).dtype).pin_memory()
+                 for name in wl.e2e_out} for _ in sets]
+    s_h2d, s_call, s_d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [torch.cuda.Event() for _ in sets] for k in ("h2d", "call", "d2h")}
+    used = [False, False]
+
+    def step(i):
+        k = i % 2
+        w = sets[k]
+        with torch.cuda.stream(s_h2d):
+            if used[k]:
+                s_h2d.wait_event(ev["call"][k])  # the previous call on this set has read its inputs
+            for name in w.e2e_in:
+                getattr(w, name).copy_(host_in[name], non_blocking=True)
+            ev["h2d"][k].record(s_h2d)
+        s_call.wait_event(ev["h2d"][k])
+        if used[k]:
+            s_call.wait_event(ev["d2h"][k])  # the previous result of this set has left the device
+        w.call(lam, stream=s_call)
+        ev["call"][k].record(s_call)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev["call"][k])
+            for name in w.e2e_out:
+                host_out[k][name].copy_(getattr(w, name), non_blocking=True)
+            ev["d2h"][k].record(s_d2h)
+        used[k] = True
+
+    for i in range(max(2, warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_h2d)
+    s_call.wait_event(a)
+    s_d2h.wait_event(a)
+    for i in range(steps):
+        step(i)
+    s_d2h.wait_event(ev["call"][(steps - 1) % 2])
+    b.record(s_d2h)  # after every copy out, which follows every call and copy in
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    skipped = int(wl.count.item())
+    hb, db = wl.host_bytes()
+    return ms, skipped, hb, db
+
+
+def _e2e_serial(wl, lam, steps, warmup):
     import torch
 
     hq, hk = to_pinned(wl.inp.q), to_pinned(wl.inp.k)

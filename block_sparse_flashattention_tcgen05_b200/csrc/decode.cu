@@ -50,7 +50,7 @@ struct DecodeSmemTail {
     uint64_t k_empty[8];
     uint64_t v_full[8];
     uint64_t v_empty[8];
-    float red[2][kConsumerWarps][16];
+    float red[2][kConsumerWarps][16];  // 16-byte aligned: read as float4
     float lred[kConsumerWarps][16];
     float rred[kConsumerWarps][16];
     float mfin[16];
@@ -442,9 +442,13 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
         if (!F8 && !mbar_wait(&tl->k_full[slot], (e / NK) & 1, &tl->abort)) set_timeout(tl, p.status);
         const uint8_t *kb = kring + slot * SB;
 
-        float acc[NT][4];
+        // two independent accumulation chains (even and odd 16-column steps of d), added at the
+        // end: half the dependent mma latency per block
+        float acc[NT][4], acc2[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) acc[nt][i] = acc2[nt][i] = 0.f;
         if constexpr (F8) {
             const uint8_t *ks_ = slices + (warp * 2 + (e & 1)) * kSliceBytes;  // converted ahead
             const int mi = lane >> 3, ri = lane & 7;
@@ -455,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
                 uint32_t a[4];
                 ldsm_x4(smem_addr(ks_ + (chunk >> 3) * kSliceBoxBytes + swz128(r, chunk & 7)), a[0], a[1], a[2], a[3]);
 #pragma unroll
-                for (int nt = 0; nt < NT; nt++) mma_f16_16816(acc[nt], a, qf[ks][nt]);
+                for (int nt = 0; nt < NT; nt++) mma_f16_16816((ks & 1) ? acc2[nt] : acc[nt], a, qf[ks][nt]);
             }
         } else {
             const int mi = lane >> 3, ri = lane & 7;
@@ -466,11 +470,15 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
                 uint32_t a[4];
                 ldsm_x4(smem_addr(kb + (chunk >> 3) * kBoxBytes + swz128(key, chunk & 7)), a[0], a[1], a[2], a[3]);
 #pragma unroll
-                for (int nt = 0; nt < NT; nt++) mma_bf16_16816(acc[nt], a, qf[ks][nt]);
+                for (int nt = 0; nt < NT; nt++) mma_bf16_16816((ks & 1) ? acc2[nt] : acc[nt], a, qf[ks][nt]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&tl->k_empty[slot]);
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) acc[nt][i] += acc2[nt][i];
 
         // scaled, masked scores in log2 units; my keys: lo = g4, hi = g4 + 8
         const int key_lo = j * kDecodeBlockN + warp * 16 + g4;
@@ -514,15 +522,31 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
             continue;
         }
 
-        // block row maxima of the whole tile, running max after the block, gap
+        // block row maxima of the whole tile (four warps' partial maxima, read as float4),
+        // running max after the block, gap
+        float mtc[NC];
+#pragma unroll
+        for (int c4 = 0; c4 < NC / 4; c4++) {
+            float4 v = *reinterpret_cast<const float4 *>(&tl->red[e & 1][0][4 * c4]);
+#pragma unroll
+            for (int w = 1; w < kConsumerWarps; w++) {
+                const float4 u = *reinterpret_cast<const float4 *>(&tl->red[e & 1][w][4 * c4]);
+                v.x = fmaxf(v.x, u.x);
+                v.y = fmaxf(v.y, u.y);
+                v.z = fmaxf(v.z, u.z);
+                v.w = fmaxf(v.w, u.w);
+            }
+            mtc[4 * c4] = v.x;
+            mtc[4 * c4 + 1] = v.y;
+            mtc[4 * c4 + 2] = v.z;
+            mtc[4 * c4 + 3] = v.w;
+        }
         float Mn[NC];
         float gap = NEG_INF;
         bool visited = false;
 #pragma unroll
         for (int c = 0; c < NC; c++) {
-            float mt = tl->red[e & 1][0][c];
-#pragma unroll
-            for (int w = 1; w < kConsumerWarps; w++) mt = fmaxf(mt, tl->red[e & 1][w][c]);
+            const float mt = mtc[c];
             Mn[c] = fmaxf(Mall[c], mt);
             if (mt > NEG_INF) {
                 visited = true;

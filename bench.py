@@ -461,6 +461,15 @@ class DecodeMqa(Decode):
     kind = "decode_mqa"
 
 
+class DecodeMqaSeeded(DecodeMqa):
+    """The same MQA decode with split seeding (splits after the first start their running
+    max at block 0's row maxima), which lifts the cap that 16 restarted splits put on its
+    sparsity.  Effective bytes as for the MQA decode (the extra block-0 reads are overhead)."""
+
+    kind = "decode_mqa_seeded"
+    seed_splits = True
+
+
 class DecodePaged:
     """Decode over a paged, ragged cache: the batch-32 GQA decode's keys, each
     sequence cut to its own length (uniform in [min_len, Lk], seeded) and
@@ -916,7 +925,8 @@ def oracle_sample(wl_kind, cfg, lam_target=0.75, budget_s=10.0, seed_tiles=0):
         inp = synth.planted_decode(c["B"], c["Hq"], c["Hkv"], c["Lk"], c["d"], seed=c["seed"], reading="blk")
         cand = list(range(c["B"] * c["Hkv"]))
         rng.shuffle(cand)
-        kw = dict(scale=inp.scale, causal=False, is_decode=True, num_splits=c["splits"])
+        kw = dict(scale=inp.scale, causal=False, is_decode=True, num_splits=c["splits"],
+                  seed_splits=c.get("seed_splits", False))
         blk = 64 * c["d"] * 2
         keyb = c["Lk"] * c["d"] * 2
         n_tiles = len(cand)
@@ -1227,6 +1237,10 @@ def main():
                                               min_len=min(8192, wls["decode"].cfg["Lk"] // 4))
         if not args.no_mqa and "decode_mqa" not in wls:
             wls["decode_mqa"] = DecodeMqa(mqa_cfg(args.size, dcfg), dev)
+        if not args.no_mqa and not args.no_seeded and "decode_mqa" in wls:
+            wm = DecodeMqaSeeded.__new__(DecodeMqaSeeded)  # shares the MQA workload's inputs and buffers
+            wm.__dict__.update(wls["decode_mqa"].__dict__)
+            wls["decode_mqa_seeded"] = wm
         if "mla" not in wls and not args.no_mla:
             wls["mla"] = Mla(mcfg, dev)
         if "prefill" in wls and "backward" not in wls and not args.no_backward:

@@ -283,13 +283,12 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     // tiles of up to 16 rows: mma.sync kernel; 17..128 rows (MQA, large groups): tcgen05 kernel
     const bool wide = R > 16;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
-    if (wide && op.seed_splits) return BLASST_ERR_UNSUPPORTED;
     int S = 0;
     st = decode_split_count(d, op.num_splits, B, Hkv, Lk, &S);
     if (st != BLASST_OK) return st;
     if (S > 65535) return BLASST_ERR_INVALID;
-    if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + S - 1) / S > 1024)
-        return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 blocks per split
+    if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + S - 1) / S > (op.seed_splits ? 1023 : 1024))
+        return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 ring entries per split (seed block included)
     if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;
     const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
     const int per_split = (nb + S - 1) / S;

@@ -20,6 +20,9 @@
 // alternate between the two P buffers, so the softmax writes P(k) once the P.V of
 // kept block k-2 (not k-1) is done: two V loads stay in flight behind the
 // decisions instead of one.
+// Seeded splits: every split after the first scores block 0 ahead of its own
+// blocks; that block's row maxima start the split's running max (no decision,
+// no exp, no P.V, nothing reported), and the split has no forced first block.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -37,7 +40,7 @@ constexpr int kBoxBytesKV = kBN * 128;     // 64 keys x 64 bf16
 constexpr int kStageBytes = 2 * kBoxBytesKV;
 constexpr int kQBytes = 2 * kBoxBytesQ;
 constexpr int kNK = 2, kNV = 2;   // two CTAs per SM: each keeps two blocks of K and of V in flight
-constexpr int kMaxWideBlocks = 1024;  // blocks per split (decision array)
+constexpr int kMaxWideBlocks = 1024;  // ring entries per split, seed block included (decision array)
 constexpr uint32_t kColP = 64, kColO = 128;  // P buffer b at kColP + 32 b
 constexpr int kDecRing = 8;                    // decisions published ahead of the MMA thread
 constexpr float kRescaleThreshold = 8.0f;
@@ -104,6 +107,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int j1 = min(nbs, j0 + per_split);
     const int nblk = max(0, j1 - j0);
     const int bh = b * p.Hkv + hkv;
+    // ring entries: [block 0 (seed)], then the split's blocks j0 .. j1-1
+    const int seed = (p.seed && split > 0 && nblk > 0) ? 1 : 0;
+    const int nent = nblk + seed;
+    auto entry_block = [&](int e) { return (seed && e == 0) ? 0 : j0 + e - seed; };
 
     if (threadIdx.x == 0) {
         mbar_init(&tl->q_full, 1);
@@ -147,13 +154,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             tma_load_3d(sq, &tmap_q, &tl->q_full, 0, qrow, b);
             tma_load_3d(sq + kBoxBytesQ, &tmap_q, &tl->q_full, 64, qrow, b);
             int issued = 0;
-            for (int jj = 0; jj < nblk && !tl->abort; jj++) {
+            for (int jj = 0; jj < nent && !tl->abort; jj++) {
                 const int st = jj % kNK;
                 if (jj >= kNK && !mbar_wait(&tl->k_empty[st], ((jj / kNK) & 1) ^ 1, &tl->abort)) {
                     set_timeout(tl, p.status);
                     break;
                 }
-                const int2 cr = block_coord(p, b, hkv, j0 + jj);
+                const int2 cr = block_coord(p, b, hkv, entry_block(jj));
                 mbar_arrive_expect_tx(&tl->k_full[st], kStageBytes);
                 tma_load_3d(sk + st * kStageBytes, &tmap_k, &tl->k_full[st], 0, cr.x, cr.y);
                 tma_load_3d(sk + st * kStageBytes + kBoxBytesKV, &tmap_k, &tl->k_full[st], 64, cr.x, cr.y);
@@ -168,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!CALIB && lane == 0 && nblk > 0) {
             tma_prefetch_desc(&tmap_v);
             int vk = 0;
-            for (int jj = 0; jj < nblk && !tl->abort; jj++) {
+            for (int jj = 0; jj < nent && !tl->abort; jj++) {
                 long long t0 = clock64();
                 while (*reinterpret_cast<volatile int *>(&tl->dec_count) <= jj) {
                     if (tl->abort || clock64() - t0 > kWaitLimitCycles) {
@@ -185,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     set_timeout(tl, p.status);
                     break;
                 }
-                const int2 cr = block_coord(p, b, hkv, j0 + jj);
+                const int2 cr = block_coord(p, b, hkv, entry_block(jj));
                 mbar_arrive_expect_tx(&tl->v_full[st], kStageBytes);
                 tma_load_3d(sv + st * kStageBytes, &tmap_v, &tl->v_full[st], 0, cr.x, cr.y);
                 tma_load_3d(sv + st * kStageBytes + kBoxBytesKV, &tmap_v, &tl->v_full[st], 64, cr.x, cr.y);
@@ -221,9 +228,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             // np's decision as it arrives (P.V when kept, then its V stage back)
             int n_pv = 0, ns = 0, np = 0, vk = 0;
             long long t_last = clock64();
-            while (ok && np < nblk) {
+            while (ok && np < nent) {
                 bool did = false;
-                if (ns < nblk && (ns == 0 || mbar_test_wait(&tl->s_free, (ns - 1) & 1)) &&
+                if (ns < nent && (ns == 0 || mbar_test_wait(&tl->s_free, (ns - 1) & 1)) &&
                     mbar_test_wait(&tl->k_full[ns % kNK], (ns / kNK) & 1)) {
                     tc_fence_after();
                     issue_s(ns);
@@ -273,12 +280,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float NEG_INF = -CUDART_INF_F;
         float m_true = NEG_INF, m_ref = NEG_INF, l = 0.f, lr = 0.f;
         int n_kept = 0;
-        bool seen = false;
+        bool seen = seed != 0;  // a seeded split has no forced first block
         unsigned int n_skip = 0;
         uint32_t mword = 0;
         int mword_idx = -1;
-        for (int jj = 0; jj < nblk; jj++) {
-            const int j = j0 + jj;
+        for (int jj = 0; jj < nent; jj++) {
+            const int j = entry_block(jj);
             const int sl = jj % kDecRing;
             if (!mbar_wait(&tl->s_full, jj & 1, &tl->abort)) set_timeout(tl, p.status);
             tc_fence_after();
@@ -308,6 +315,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                 m3 = fmax3(m3, s[c + 6], s[c + 7]);
             }
             const float mt = fmax3(m0, m1, fmaxf(m2, m3)) * p.scale_log2;
+            // the MMA thread has taken the decision published kDecRing entries ago
+            if (jj >= kDecRing && !mbar_wait(&tl->dec_free[sl], ((jj / kDecRing) - 1) & 1, &tl->abort))
+                set_timeout(tl, p.status);
+            if (seed && jj == 0) {
+                // the seed block: its row maxima start the running max of this split
+                m_true = mt;
+                if (row == 0) {
+                    dec[jj] = 0;
+                    __threadfence_block();
+                    *reinterpret_cast<volatile int *>(&tl->dec_count) = jj + 1;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tl->p_full[sl]);
+                continue;
+            }
             const float mn = fmaxf(m_true, mt);
             const bool vote = (mt == NEG_INF) || (mt - mn < p.thr_log2);
             const bool all = bar_and(1, 128, vote);
@@ -318,9 +340,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             seen = seen || visited;
             const bool skip = visited && all && !first;
             const bool kept = visited && !skip;
-            // the MMA thread has taken the decision published kDecRing blocks ago
-            if (jj >= kDecRing && !mbar_wait(&tl->dec_free[sl], ((jj / kDecRing) - 1) & 1, &tl->abort))
-                set_timeout(tl, p.status);
             if (row == 0) {
                 // the V producer reads the decision before this block's exponentials run
                 dec[jj] = kept ? 1 : 0;

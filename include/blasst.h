@@ -96,7 +96,7 @@ typedef struct blasst_opts {
                                   tile's (split's) first block, NaN if not visited */
     unsigned int *status_word; /* device word the caller zeroes; the library ORs in
                                   a nonzero code when a bounded wait expires */
-    int seed_splits;           /* decode only (d = 128 tiles of up to 16 rows, and MLA):
+    int seed_splits;           /* decode only (d = 128 tiles of any width, and MLA):
                                   nonzero seeds the running
                                   max of every split after the first with the row
                                   maxima of block 0, and such a split has no forced
@@ -124,8 +124,8 @@ BLASST_API blasst_status blasst_prefill(const void *q, const void *k, const void
 /*
  * Decode: the G = Hq/Hkv query heads x Lq queries of one KV head form the
  * tile (G * Lq <= 128; up to 16 rows on mma.sync, 17 to 128 rows -- MQA with
- * many heads, large GQA groups -- on tcgen05 with the tile in tensor memory;
- * seed_splits only up to 16 rows), KV blocks of 64 keys, split-KV over num_splits
+ * many heads, large GQA groups -- on tcgen05 with the tile in tensor memory),
+ * KV blocks of 64 keys, split-KV over num_splits
  * contiguous chunks of ceil(n_blocks / num_splits) blocks.  Each split is an
  * independent online-softmax pass (running max restarts, its first block is
  * kept); the skip decision for a block is taken after its K block is read and

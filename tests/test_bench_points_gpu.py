@@ -59,6 +59,10 @@ def workload(name, dev):
             wl.__dict__.update(src.__dict__)
         elif name == "decode_mqa":
             wl = bench.DecodeMqa(bench.MQA, dev)
+        elif name == "decode_mqa_seeded":
+            src = workload("decode_mqa", dev)[0]
+            wl = bench.DecodeMqaSeeded.__new__(bench.DecodeMqaSeeded)
+            wl.__dict__.update(src.__dict__)
         elif name == "mla":
             wl = bench.Mla(bench.MLA, dev)
         elif name == "decode_paged":
@@ -133,7 +137,7 @@ def _decode_check(inp, lam, splits, o, lse, mask, tiles, seed_splits=False, k=No
     return bits
 
 
-@pytest.mark.parametrize("name", ["decode", "decode_seeded", "decode_mqa"])
+@pytest.mark.parametrize("name", ["decode", "decode_seeded", "decode_mqa", "decode_mqa_seeded"])
 @pytest.mark.parametrize("target", TARGETS)
 def test_decode_at_bench_lambda(dev, name, target):
     import block_sparse_flashattention_tcgen05_b200 as bl

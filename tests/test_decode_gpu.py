@@ -290,6 +290,52 @@ def test_decode_seeded_skips_contain_unseeded(bl):
     assert int(c1.item()) > int(c0.item())
 
 
+# seeded splits on wide tiles (the tcgen05 decode)
+@pytest.mark.parametrize("lam", [0.0, 1e-3, 0.05, 0.5, 0.999])
+@pytest.mark.parametrize("splits", [4, 16])
+def test_decode_mqa_seeded(bl, lam, splits):
+    inp = planted_decode(2, 32, 1, 64 * 41 + 13, 128, seed=51, reading="blk")
+    bits, _ = check_decode(bl, inp, lam, False, splits, seed_splits=True)
+    if lam == 0.0:
+        assert bits.sum() == 0
+
+
+def test_decode_wide_seeded_causal_two_queries(bl):
+    inp = planted_decode(1, 64, 1, 2500, 128, Lq=2, seed=54, reading="blk")
+    check_decode(bl, inp, 0.1, True, 5, seed_splits=True)
+
+
+def test_decode_wide_seeded_short_cache_empty_splits(bl):
+    inp = planted_decode(2, 32, 1, 90, 128, seed=55, reading="lit")
+    check_decode(bl, inp, 0.3, False, 16, seed_splits=True)
+
+
+def test_decode_wide_seeded_calibrate_gaps(bl):
+    inp = planted_decode(2, 64, 2, 3000, 128, seed=56, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    gaps, mc, cc = bl.calibrate(q, k, scale=inp.scale, lam=0.05, mode="decode", num_splits=6, seed_splits=True)
+    _, _, md, cd = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=6, seed_splits=True)
+    torch.cuda.synchronize()
+    assert torch.equal(mc, md) and torch.equal(cc, cd)
+    ref = oracle.attention(inp.q, inp.k, inp.v, scale=inp.scale, lam=0.05, causal=False, is_decode=True,
+                           num_splits=6, BN=64, seed_splits=True)
+    g = gaps.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(ref["gaps"])
+    assert np.array_equal(np.isinf(g), np.isinf(ref["gaps"]))
+    assert np.max(np.abs(g[fin] - ref["gaps"][fin])) < 1e-3
+
+
+def test_decode_wide_seeded_skips_contain_unseeded(bl):
+    inp = planted_decode(2, 128, 1, 8192, 128, seed=58, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    _, _, m0, c0 = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=16)
+    _, _, m1, c1 = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=16, seed_splits=True)
+    torch.cuda.synchronize()
+    a, b = m0.cpu().numpy().astype(np.uint32), m1.cpu().numpy().astype(np.uint32)
+    assert np.all((a & ~b) == 0)
+    assert int(c1.item()) > int(c0.item())
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("lam", [0.0, 0.05])
 def test_decode_seeded_full_size_sampled(bl, lam):

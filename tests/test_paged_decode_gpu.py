@@ -115,6 +115,13 @@ def test_paged_mqa_wide_tile(bl):
     check_paged(bl, inp, [2600, 65, 1300], 0.05, 4)
 
 
+@pytest.mark.parametrize("lam", [0.0, 0.05])
+def test_paged_mqa_wide_tile_seeded(bl, lam):
+    # seeded splits on the tcgen05 decode over ragged pages (one sequence shorter than a split)
+    inp = planted_decode(3, 64, 1, 2600, 128, seed=38, reading="blk")
+    check_paged(bl, inp, [2600, 65, 1300], lam, 6, seed_splits=True)
+
+
 def test_paged_single_key_sequences(bl):
     inp = planted_decode(3, 4, 1, 200, 128, seed=34, reading="lit")
     check_paged(bl, inp, [1, 63, 200], 0.3, 16)

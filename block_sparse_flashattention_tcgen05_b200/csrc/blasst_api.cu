@@ -198,7 +198,9 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
         e = cudaMemsetAsync(skip_mask, 0, (size_t)B * words * sizeof(uint32_t), sm);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_mask)");
     }
-    if (skip_count) {
+    // the calibration pass adds into skip_count; an attention call's split CTAs store their
+    // counts in the workspace and the combine kernel writes the sum (no reset needed)
+    if (skip_count && calib) {
         e = cudaMemsetAsync(skip_count, 0, sizeof(unsigned long long), sm);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_count)");
     }
@@ -208,7 +210,11 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
     p.part_o = calib ? nullptr : static_cast<float *>(ws);
     p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));
     p.skip_mask = skip_mask;
-    p.skip_count = skip_count;
+    p.skip_count = calib ? skip_count : nullptr;
+    p.split_skips = (calib || !skip_count) ? nullptr
+                                           : reinterpret_cast<unsigned int *>(static_cast<char *>(ws) +
+                                                                              round_up(rows * S * c.dv * 4, 256) +
+                                                                              round_up(rows * S * 4, 256));
     p.gaps = op.gaps_out;
     p.status = op.status_word;
     p.B = B; p.Hq = Hq; p.Lq = Lq; p.Lk = Lk; p.R = (int)R;
@@ -228,6 +234,9 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
         cp.rows = (int)rows;
         cp.num_splits = S;
         cp.dv = c.dv;
+        cp.split_skips = p.split_skips;
+        cp.n_counts = B * S;
+        cp.skip_count = skip_count;
         e = launch_combine(cp, sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel");
     }
@@ -290,6 +299,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + S - 1) / S > (op.seed_splits ? 1023 : 1024))
         return BLASST_ERR_UNSUPPORTED;  // wide tiles: at most 1024 ring entries per split (seed block included)
     if (Hkv > 65535 || B > 65535) return BLASST_ERR_UNSUPPORTED;
+    if ((long long)S * Hkv * B > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED;  // one CTA (and count slot) per split
     const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
     const int per_split = (nb + S - 1) / S;
     if (per_split > kMaxBlocksPerSplit) return BLASST_ERR_UNSUPPORTED;
@@ -339,7 +349,9 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         e = cudaMemsetAsync(skip_mask, 0, (size_t)B * Hkv * words * sizeof(uint32_t), sm);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_mask)");
     }
-    if (skip_count) {
+    // the calibration pass adds into skip_count; an attention call's split CTAs store their
+    // counts in the workspace and the combine kernel writes the sum (no reset needed)
+    if (skip_count && calib) {
         e = cudaMemsetAsync(skip_count, 0, sizeof(unsigned long long), sm);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(skip_count)");
     }
@@ -350,7 +362,11 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     p.part_o = calib ? nullptr : static_cast<float *>(ws);
     p.part_lse = calib ? nullptr : reinterpret_cast<float *>(static_cast<char *>(ws) + round_up(rows * S * c.dv * 4, 256));
     p.skip_mask = skip_mask;
-    p.skip_count = skip_count;
+    p.skip_count = calib ? skip_count : nullptr;
+    p.split_skips = (calib || !skip_count) ? nullptr
+                                           : reinterpret_cast<unsigned int *>(static_cast<char *>(ws) +
+                                                                              round_up(rows * S * c.dv * 4, 256) +
+                                                                              round_up(rows * S * 4, 256));
     p.gaps = op.gaps_out;
     p.status = op.status_word;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.G = G; p.R = (int)R;
@@ -382,6 +398,9 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
         cp.rows = (int)rows;
         cp.num_splits = S;
         cp.dv = c.dv;
+        cp.split_skips = p.split_skips;
+        cp.n_counts = S * Hkv * B;
+        cp.skip_count = skip_count;
         e = launch_combine(cp, sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode combine kernel");
     }
@@ -671,7 +690,8 @@ size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_spli
     const size_t S = num_splits ? num_splits : 16;
     const size_t rows = (size_t)B * Hq * Lq;
     const size_t dvv = dv ? dv : 128;
-    return round_up(rows * S * dvv * 4, 256) + round_up(rows * S * 4, 256);
+    // partial O, partial lse, then one skip-count slot per split CTA (at most B * Hq * S)
+    return round_up(rows * S * dvv * 4, 256) + round_up(rows * S * 4, 256) + round_up((size_t)B * Hq * S * 4, 256);
 }
 
 long long blasst_visited_pairs(int B, int Hq, int Hkv, int Lq, int Lk, int causal, int is_decode,

@@ -622,7 +622,10 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
     if (warp == 0 && lane == 0) {
         if (p.skip_mask && mask_word_idx >= 0 && mask_word)
             atomicOr(p.skip_mask + (size_t)bh * p.words + mask_word_idx, mask_word);
-        if (p.skip_count && n_skip) atomicAdd(p.skip_count, n_skip);
+        if (p.split_skips)
+            p.split_skips[blockIdx.x] = (unsigned int)n_skip;
+        else if (p.skip_count && n_skip)
+            atomicAdd(p.skip_count, n_skip);
     }
     if (CALIB) return;
 
@@ -678,8 +681,20 @@ __global__ void __launch_bounds__(kThreads, (F8 && NT == 1) ? 2 : 1)
 
 // One warp per output row: lse = ln sum_s exp(lse_s); O = sum_s exp(lse_s - lse) O_s.
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+    pdl_wait();  // the split kernel has finished and its partials are visible
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
+    if (p.skip_count && blockIdx.x == 0) {
+        // the split CTAs' skip counts, one slot each: their sum is the call's count
+        __shared__ unsigned long long part[4];
+        unsigned long long s = 0;
+        for (int i = threadIdx.x; i < p.n_counts; i += 128) s += p.split_skips[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) part[threadIdx.x >> 5] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) *p.skip_count = part[0] + part[1] + part[2] + part[3];
+    }
     if (row >= p.rows) return;
     const int S = p.num_splits;
     const float LOG2E = 1.4426950408889634f;
@@ -741,8 +756,21 @@ cudaError_t launch_decode_fp8(const DecodeParams &p, const CUtensorMap &tk, cons
 
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t st) {
     if (p.rows == 0) return cudaSuccess;
-    combine_kernel<<<(p.rows + 3) / 4, 128, 0, st>>>(p);
-    return cudaGetLastError();
+    // programmatic dependent launch: the combine's launch is processed while the split
+    // kernel runs, and its CTAs start as the split CTAs exit, each waiting on the device
+    // (griddepcontrol.wait) for the split grid's completion and memory.  (An explicit early
+    // signal from the split CTAs, at their start, measured slower.)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((p.rows + 3) / 4);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 }  // namespace blasst

@@ -431,7 +431,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (row == 0) {
             if (p.skip_mask && mword_idx >= 0 && mword) atomicOr(p.skip_mask + (size_t)bh * p.words + mword_idx, mword);
-            if (p.skip_count && n_skip) atomicAdd(p.skip_count, (unsigned long long)n_skip);
+            if (p.split_skips)
+                p.split_skips[(size_t)bh * p.num_splits + split] = n_skip;
+            else if (p.skip_count && n_skip)
+                atomicAdd(p.skip_count, (unsigned long long)n_skip);
         }
         if (!CALIB) {
             // split epilogue: normalised partial O and the split's lse for each valid row

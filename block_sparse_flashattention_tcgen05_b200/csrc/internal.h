@@ -20,7 +20,9 @@ struct DecodeParams {
     float *part_o;                  // [B*Hq*Lq, S, dv] fp32 split outputs (normalised)
     float *part_lse;                // [B*Hq*Lq, S] fp32 split lse (natural log)
     uint32_t *skip_mask;            // [B, Hkv, 1, W] or null
-    unsigned long long *skip_count; // or null
+    unsigned long long *skip_count; // or null: every CTA adds its skipped blocks (calibration pass)
+    unsigned int *split_skips;      // or null: every CTA stores its skipped blocks in its own slot
+                                    // (attention calls; the combine kernel sums the slots)
     float *gaps;                    // [B*Hkv, nb] or null
     unsigned int *status;           // or null
     int B, Hq, Hkv, Lq, Lk, G, R;   // R = G * Lq rows per tile
@@ -45,6 +47,9 @@ struct CombineParams {
     int rows;         // B * Hq * Lq
     int num_splits;
     int dv;
+    const unsigned int *split_skips;  // per-CTA skip counts of the split kernel, or null
+    int n_counts;                     // slots in split_skips
+    unsigned long long *skip_count;   // their sum is stored here (when not null)
 };
 
 // One prefill (or prefill-shaped calibration) call.
@@ -85,7 +90,8 @@ struct MlaParams {
     float *part_o;                  // [B*Hq*Lq, S, 512] fp32 split outputs (normalised)
     float *part_lse;                // [B*Hq*Lq, S]
     uint32_t *skip_mask;            // [B, 1, 1, W] or null
-    unsigned long long *skip_count; // or null
+    unsigned long long *skip_count; // or null (calibration pass: added to)
+    unsigned int *split_skips;      // [B, S] or null (attention calls: one slot per split)
     float *gaps;                    // [B, nb] or null
     unsigned int *status;           // or null
     int B, Hq, Lq, Lk, R;           // R = Hq * Lq <= 128

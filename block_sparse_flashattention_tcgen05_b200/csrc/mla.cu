@@ -396,7 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (row == 0 && report) {
             if (p.skip_mask && mword_idx >= 0 && mword) atomicOr(p.skip_mask + (size_t)b * p.words + mword_idx, mword);
-            if (p.skip_count && n_skip) atomicAdd(p.skip_count, (unsigned long long)n_skip);
+            if (p.split_skips)
+                p.split_skips[(size_t)b * p.num_splits + split] = n_skip;
+            else if (p.skip_count && n_skip)
+                atomicAdd(p.skip_count, (unsigned long long)n_skip);
         }
         if (!CALIB) {
             // split epilogue: normalised partial O (this CTA's 256 value columns), the split's lse
@@ -437,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 256; i += 4) *reinterpret_cast<float4 *>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
             if (half == 0) p.part_lse[orow] = -CUDART_INF_F;
         }
+        if (half == 0 && threadIdx.x == 0 && p.split_skips) p.split_skips[(size_t)b * p.num_splits + split] = 0;
     }
     tc_fence_before();
     __syncthreads();

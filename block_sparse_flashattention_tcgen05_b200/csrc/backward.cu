@@ -11,8 +11,9 @@
 //   main      one CTA per (KV block j of 128 keys, KV head, sequence) walks the
 //             kept (query tile i, query head) pairs of its KV head in order
 //             and accumulates dK_j and dV_j over all of them in tensor memory;
-//             dQ_i contributions go to the fp32 accumulator by coalesced
-//             red.add (each warp adds 128 contiguous bytes of one query row);
+//             dQ_i contributions go to the fp32 accumulator by bulk reduce-add
+//             (cp.reduce.async.bulk .add.f32, two 32 KB row ranges per pair)
+//             from shared memory, staged by the compute warps;
 //   finalize  dQ accumulator -> bf16 dq.
 //
 // Main kernel, per pair (S^T etc. are key-major: TMEM lane = key of block j):
@@ -30,18 +31,24 @@
 //              kColGroups columns);
 //   producer   TMA: K_j, V_j once; Q_i, dO_i and the two per-row vectors per
 //              pair into a 2-stage ring;
-//   MMA        allocates TMEM and issues every tcgen05.mma from one thread.
+//   MMA        allocates TMEM and issues every tcgen05.mma from one thread;
+//   reduce     issues the bulk reduce-add of each pair's staged dQ rows.
 //
 // TMEM (512 columns): S^T [0,128) -> P^T (bf16; each column group's P^T packed
 // into the first half of its own S^T columns); dP^T [128,256) -> dQ^T;
 // dV [256,384); dK [384,512).
 //
 // MMA issue order per pair t: dP(t) [after the dQ^T(t-1) columns are read],
-// then, once dS^T(t) is ready: dQ^T(t), dV(t), S(t+1), dK(t) -- or dK(t)
-// before S(t+1) when pair t+1's Q tile has not landed yet.  The compute warps
-// form P(t+1) from S(t+1) while dK(t) and dP(t+1) run.  Operations issued by
-// one thread execute in issue order, so S(t+1) overwrites P^T(t) only after
-// dV(t) has read it, and a commit covers every earlier operation.
+// then, once dS^T(t) is ready: dQ^T(t), dK(t), dV(t), S(t+1).  Operations
+// issued by one thread execute in issue order, so S(t+1) overwrites P^T(t) only
+// after dV(t) has read it, and a commit covers every earlier operation.
+// dQ staging: once dK(t) has completed, neither Q(t)'s stage nor the dS^T
+// buffer is read again, and they take dQ(t) as fp32 rows (queries 0-63 in the
+// Q stage, 64-127 in the dS^T buffer, 512 bytes of head dims per row, the
+// accumulator's own layout) while the tensor core runs dV(t) and S(t+1).  The
+// reduce warp adds both ranges to the accumulator and returns the buffers
+// (stage_free) once the bulk copies have read them: the dS^T buffer to the
+// compute warps for dS(t+1), the Q stage to the producer for pair t+2.
 #include <climits>
 
 #include <cuda_bf16.h>
@@ -64,7 +71,8 @@ constexpr int kChunks = kCW / 32;      // 32-column TMEM loads per operand
 constexpr int kComputeWarps = 4 * kColGroups;
 constexpr int kProducerWarp = kComputeWarps;
 constexpr int kMmaWarp = kComputeWarps + 1;
-constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kReduceWarp = kComputeWarps + 2;
+constexpr int kThreads = 32 * (kComputeWarps + 3);
 static_assert(kColGroups == 2 || kColGroups == 4, "64 or 32 columns per compute warp");
 constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
 constexpr int kBoxBytes = kTileBytes / 2;  // 128 rows x 64 bf16 (one 128-byte swizzle box)
@@ -77,6 +85,9 @@ struct BwdTail {
     uint64_t kv_full;
     uint64_t qdo_full[2], qdo_empty[2];
     uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
+    uint64_t dk_done;        // dK(t) done: Q(t)'s stage and the dS^T buffer are free for dQ(t)
+    uint64_t dq_staged;      // the compute warps have written dQ(t) rows to them
+    uint64_t stage_free[2];  // [Q stage]: the bulk reduce of dQ(t) has read the staged rows
     uint32_t tmem_base;
     int abort;
 };
@@ -161,6 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&tl->dq_full, 1);
         mbar_init(&tl->dq_free, kComputeWarps);
         mbar_init(&tl->acc_done, 1);
+        mbar_init(&tl->dk_done, 1);
+        mbar_init(&tl->dq_staged, kComputeWarps);
+        mbar_init(&tl->stage_free[0], 1);
+        mbar_init(&tl->stage_free[1], 1);
         tl->abort = 0;
         fence_mbar_init();
     }
@@ -189,7 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             int i = first_tile(p, j), g = 0, t = 0;
             while (!tl->abort && next_pair(p, b, hkv, j, i, g)) {
                 const int st = t & 1;
-                if (t >= 2 && !mbar_wait(&tl->qdo_empty[st], ((t >> 1) & 1) ^ 1, &tl->abort)) {
+                // the stage held pair t-2: the tensor core is done with it and the dQ rows staged
+                // in its Q tile have been read by the bulk reduce
+                if (t >= 2 && (!mbar_wait(&tl->qdo_empty[st], ((t >> 1) & 1) ^ 1, &tl->abort) ||
+                               !mbar_wait(&tl->stage_free[st], ((t >> 1) & 1) ^ 1, &tl->abort))) {
                     set_timeout(tl, p.status);
                     break;
                 }
@@ -278,27 +296,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < 8; kk++)
                     umma_ss2(tmem + 128, k_mn + kk * (2048 >> 4), ds_mn + kk * (2048 >> 4), dhi, idesc_mnmn, kk > 0);
                 umma_commit(&tl->dq_full);
+                // dK += dS^T Q (K = 128 queries); then Q(t)'s stage and the dS^T buffer take dQ(t)
+#pragma unroll
+                for (int kk = 0; kk < 8; kk++)
+                    umma_ss2(tmem + 384, ds_km + koff(kk), q_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn,
+                             (t > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&tl->dk_done);
                 // dV += P^T dO (K = 128 queries; P^T of each column group in its own S^T columns)
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++)
                     umma_ts2(tmem + 256, tmem + (uint32_t)((kk * 16 / kCW) * kCW + (kk * 16 % kCW) / 2),
                              do_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn, (t > 0 || kk > 0) ? 1u : 0u);
-                auto issue_dk = [&]() {  // dK += dS^T Q (K = 128 queries)
-#pragma unroll
-                    for (int kk = 0; kk < 8; kk++)
-                        umma_ss2(tmem + 384, ds_km + koff(kk), q_mn + st * kStage16 + kk * (2048 >> 4), dhi,
-                                 idesc_kmn, (t > 0 || kk > 0) ? 1u : 0u);
-                };
-                // The next pair's S^T goes ahead of dK(t) when its Q tile has landed, so that its
-                // exponentials overlap dK(t) and dP(t+1); otherwise dK(t) keeps the pipe busy first.
-                bool dk_done = false;
+                umma_commit(&tl->qdo_empty[st]);
+                // the next pair's S^T (overwrites P^T(t), which dV(t) above has read)
                 if (more) {
-                    const uint32_t npar = ((t + 1) >> 1) & 1;
-                    if (!mbar_test_wait(&tl->qdo_full[nst], npar)) {
-                        issue_dk();
-                        dk_done = true;
-                    }
-                    if (!mbar_wait(&tl->qdo_full[nst], npar, &tl->abort)) {
+                    if (!mbar_wait(&tl->qdo_full[nst], ((t + 1) >> 1) & 1, &tl->abort)) {
                         set_timeout(tl, p.status);
                         break;
                     }
@@ -306,8 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issue_s(nst);
                     umma_commit(&tl->s_full);
                 }
-                if (!dk_done) issue_dk();
-                umma_commit(&tl->qdo_empty[st]);
                 t++;
                 i = ni;
                 g = ng;
@@ -315,6 +325,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // every MMA of this thread has completed: dK, dV final, TMEM free to release
             umma_commit(&tl->acc_done);
+        }
+        __syncwarp();
+    } else if (warp == kReduceWarp) {
+        // ----------------------------------------------------------- dQ bulk reduce
+        if (lane == 0) {
+            int i = first_tile(p, j), g = 0, t = 0;
+            while (!tl->abort && next_pair(p, b, hkv, j, i, g)) {
+                const int st = t & 1;
+                if (!mbar_wait(&tl->dq_staged, t & 1, &tl->abort)) {
+                    set_timeout(tl, p.status);
+                    break;
+                }
+                const int qrow = b * p.Hq + hkv * p.G + g;
+                float *dst = p.dq_acc + ((size_t)qrow * p.Lq_pad + (size_t)i * 128) * 128;
+                bulk_reduce_add_f32(dst, sQ + st * kTileBytes, 64 * 128 * 4);
+                bulk_reduce_add_f32(dst + 64 * 128, sdS, 64 * 128 * 4);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(&tl->stage_free[st]);
+                t++;
+                advance(p, i, g);
+            }
+            bulk_wait_all();  // every addition has been performed before the CTA exits
         }
         __syncwarp();
     } else {
@@ -329,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (__all_sync(0xffffffffu, !tl->abort && next_pair(p, b, hkv, j, i, g))) {
             const int st = t & 1;
             const int q0 = i * 128 + hh * kCW;  // first query row of my columns
-            const int qrow = b * p.Hq + hkv * p.G + g;
             if (!warp_wait(&tl->qdo_full[st], (t >> 1) & 1, &tl->abort) ||
                 !warp_wait(&tl->s_full, t & 1, &tl->abort)) {
                 set_timeout(tl, p.status);
@@ -374,6 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            // the dS^T buffer held dQ(t-1)'s staged rows until the bulk reduce read them
+            if (t > 0 && !warp_wait(&tl->stage_free[(t - 1) & 1], ((t - 1) >> 1) & 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
             // dS^T row r, my queries -> their 64-query box of sdS (128-byte swizzle, chunks of 8 queries)
             uint8_t *ds_row = sdS + (hh * kCW / 64) * kBoxBytes;
             const int chunk0 = (hh * kCW % 64) / 8;
@@ -419,12 +456,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tl->dq_free);
-            // a warp adds 128 contiguous bytes (32 head dims of one query row) per instruction
-            float *acc = p.dq_acc + ((size_t)qrow * p.Lq_pad + q0) * 128 + r;
-            const int nvalid = min(kCW, p.Lq - q0);
+            // stage dQ(t) once dK(t) is done: query rows of 128 fp32 head dims, rows 0-63 in
+            // Q(t)'s stage and 64-127 in the dS^T buffer (a warp store covers 128 contiguous bytes
+            // of one row); rows past Lq hold zeros (their P, hence dS, is 0)
+            if (!warp_wait(&tl->dk_done, t & 1, &tl->abort)) {
+                set_timeout(tl, p.status);
+                break;
+            }
+            float *stg = reinterpret_cast<float *>(hh * kCW < 64 ? sQ + st * kTileBytes : sdS) +
+                         ((hh * kCW) & 63) * 128 + r;
 #pragma unroll
-            for (int c = 0; c < kCW; c++)
-                if (c < nvalid) atomicAdd(acc + (size_t)c * 128, __uint_as_float(qa[c]));
+            for (int c = 0; c < kCW; c++) stg[c * 128] = __uint_as_float(qa[c]);
+            fence_proxy_async();  // the stores -> visible to the bulk copy's reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tl->dq_staged);
             t++;
             advance(p, i, g);
         }

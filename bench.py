@@ -1257,11 +1257,13 @@ def main():
         rounds = 4
         for kind, w in wls.items():
             # the sparsity points of a workload are timed round-robin, so that a drift of
-            # clocks or temperature during the sweep lands on all of them alike
+            # clocks or temperature during the sweep lands on all of them alike; odd rounds
+            # take the points in reverse order, so that no point always follows the dense one
+            # (whose power draw lowers the clock of what runs right after it)
             times = {t: [] for t in TARGETS}
             sk_by_t = {}
             for rnd in range(rounds):
-                for t in TARGETS:
+                for t in (TARGETS if rnd % 2 == 0 else TARGETS[::-1]):
                     ms_t, sk_by_t[t] = timed_launches(w, lams[kind][t][0], max(2, args.steps // (2 * rounds)),
                                                       3 if rnd == 0 else 1, flush)
                     times[t] += ms_t

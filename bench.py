@@ -49,8 +49,9 @@ PREFILL = dict(workload="prefill GQA 32K (Llama-3.1-8B attention shape)", B=1, H
 DECODE = dict(workload="decode GQA 32K cache, 16 splits", B=32, Hq=32, Hkv=8, Lk=32768, d=128, splits=16, seed=3)
 MLA = dict(workload="MLA decode, 128 heads, 576/512 latent, 32K cache, 8 seeded splits", B=64, Hq=128, Lk=32768,
            splits=8, seed_splits=True, seed=5)
-MQA = dict(workload="decode MQA, 128 query heads on one KV head, 32K cache, 16 splits", B=64, Hq=128, Hkv=1,
-           Lk=32768, d=128, splits=16, seed=9)
+# 9 splits: what num_splits=-1 picks for this 128-row tile on 148 SMs (576 CTAs, just under two waves of two per SM)
+MQA = dict(workload="decode MQA, 128 query heads on one KV head, 32K cache, 9 splits", B=64, Hq=128, Hkv=1,
+           Lk=32768, d=128, splits=9, seed=9)
 PREFILL_64K = dict(PREFILL, workload="prefill GQA 64K (Qwen3-8B-like attention shape)", L=65536, seed=4)
 QUICK_PREFILL = dict(PREFILL, workload="prefill GQA 4K (quick)", L=4096)
 QUICK_DECODE = dict(DECODE, workload="decode GQA 4K cache (quick)", B=4, Lk=4096)

@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
         L.blasst_decode_pick_splits.restype = ctypes.c_int
         L.blasst_decode_pick_splits.argtypes = [ctypes.c_int] * 4
+        L.blasst_decode_pick_splits_rows.restype = ctypes.c_int
+        L.blasst_decode_pick_splits_rows.argtypes = [ctypes.c_int] * 5
         L.blasst_decode_workspace_bytes.restype = ctypes.c_size_t
         L.blasst_decode_workspace_bytes.argtypes = [ctypes.c_int] * 5
         L.blasst_visited_pairs.restype = ctypes.c_longlong
@@ -224,13 +226,14 @@ def prefill_backward(q, k, v, o, lse, dout, *, scale, causal=True, skip_mask=Non
     return dq, dk, dv
 
 
-def decode_pick_splits(B, Hkv, Lk, num_sms=None) -> int:
-    """The split count num_splits=-1 selects (num_sms: this device's SM count by default)."""
+def decode_pick_splits(B, Hkv, Lk, num_sms=None, rows=1) -> int:
+    """The split count num_splits=-1 selects for tiles of ``rows`` = G * Lq query rows
+    (num_sms: this device's SM count by default)."""
     if num_sms is None:
         import torch
 
         num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    return int(lib().blasst_decode_pick_splits(B, Hkv, Lk, num_sms))
+    return int(lib().blasst_decode_pick_splits_rows(B, Hkv, rows, Lk, num_sms))
 
 
 def backward_workspace_bytes(B, Hq, Lq) -> int:

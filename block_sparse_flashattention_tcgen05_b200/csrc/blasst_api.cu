@@ -137,7 +137,7 @@ const double kLog2e = 1.4426950408889634;
 
 }  // namespace
 
-blasst_status blasst::decode_split_count(int d, int num_splits, int B, int Hkv, int Lk, int *out) {
+blasst_status blasst::decode_split_count(int d, int num_splits, int B, int Hkv, int rows, int Lk, int *out) {
     *out = 0;
     if (num_splits > 0) {
         *out = num_splits;
@@ -153,7 +153,7 @@ blasst_status blasst::decode_split_count(int d, int num_splits, int B, int Hkv, 
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(multiprocessors)");
-    *out = blasst_decode_pick_splits(B, Hkv, Lk, sms);
+    *out = blasst_decode_pick_splits_rows(B, Hkv, rows, Lk, sms);
     return BLASST_OK;
 }
 
@@ -170,7 +170,7 @@ blasst_status run_mla(const void *q, const void *k, const void *v, void *o, floa
     const long long R = (long long)Hq * Lq;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
     int S = 0;
-    blasst_status sst = decode_split_count(d, op.num_splits, B, Hkv, Lk, &S);
+    blasst_status sst = decode_split_count(d, op.num_splits, B, Hkv, (int)R, Lk, &S);
     if (sst != BLASST_OK) return sst;
     if (S > 65535 || B > 65535) return BLASST_ERR_INVALID;
     const int nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
@@ -293,7 +293,7 @@ blasst_status run_decode(const void *q, const void *k, const void *v, void *o, f
     const bool wide = R > 16;
     if (R > 128) return BLASST_ERR_UNSUPPORTED;
     int S = 0;
-    st = decode_split_count(d, op.num_splits, B, Hkv, Lk, &S);
+    st = decode_split_count(d, op.num_splits, B, Hkv, (int)R, Lk, &S);
     if (st != BLASST_OK) return st;
     if (S > 65535) return BLASST_ERR_INVALID;
     if (wide && ((Lk + kDecodeBlockN - 1) / kDecodeBlockN + S - 1) / S > (op.seed_splits ? 1023 : 1024))
@@ -682,6 +682,18 @@ int blasst_decode_pick_splits(int B, int Hkv, int Lk, int num_sms) {
     const long long nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
     const long long cap = std::max(1LL, std::min(64LL, nb / 32));  // at least 32 blocks per split
     const long long want = (16LL * num_sms + groups - 1) / groups;  // about 16 CTAs per SM over the call
+    return (int)std::max(1LL, std::min(cap, want));
+}
+
+int blasst_decode_pick_splits_rows(int B, int Hkv, int rows, int Lk, int num_sms) {
+    if (rows <= 16) return blasst_decode_pick_splits(B, Hkv, Lk, num_sms);
+    if (B <= 0 || Hkv <= 0 || Lk <= 0 || num_sms <= 0) return 1;
+    // wide tiles (tcgen05 kernel, two CTAs per SM): as many splits as keep the grid within two
+    // full waves of two CTAs per SM, under the same cap
+    const long long groups = (long long)B * Hkv;
+    const long long nb = (Lk + kDecodeBlockN - 1) / kDecodeBlockN;
+    const long long cap = std::max(1LL, std::min(64LL, nb / 32));
+    const long long want = 4LL * num_sms / groups;
     return (int)std::max(1LL, std::min(cap, want));
 }
 

@@ -108,7 +108,9 @@ BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, con
     // the split count and value width exactly as blasst_decode will resolve them
     // (MLA defaults to 2 splits, GQA/MQA to 16, -1 to the adaptive count)
     int splits = 0;
-    blasst_status st = blasst::decode_split_count(d, op.num_splits, B, Hkv, Lk, &splits);
+    const long long rows = (Hkv > 0 && Hq % Hkv == 0) ? (long long)(Hq / Hkv) * Lq : 0;
+    if (rows <= 0 || rows > 0x7fffffffLL) return BLASST_ERR_INVALID;
+    blasst_status st = blasst::decode_split_count(d, op.num_splits, B, Hkv, (int)rows, Lk, &splits);
     if (st != BLASST_OK) return st;
     op.num_splits = splits;
     const int dv = op.dv ? op.dv : d;

@@ -107,10 +107,11 @@ cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &tmap_q, const
                             const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, cudaStream_t stream);
 // Records the text returned by blasst_last_error() for this thread.
 void set_last_error(const char *msg);
-// The split count a decode call with these arguments uses: num_splits when positive;
-// 0 -> 16 (d = 128) or 2 (MLA, d = 576); -1 -> blasst_decode_pick_splits with the current
-// device's SM count (d = 128 only; BLASST_ERR_INVALID for MLA and other negative values).
-blasst_status decode_split_count(int d, int num_splits, int B, int Hkv, int Lk, int *out);
+// The split count a decode call with these arguments uses (rows = G * Lq, the tile's rows):
+// num_splits when positive; 0 -> 16 (d = 128) or 2 (MLA, d = 576); -1 ->
+// blasst_decode_pick_splits_rows with the current device's SM count (d = 128 only;
+// BLASST_ERR_INVALID for MLA and other negative values).
+blasst_status decode_split_count(int d, int num_splits, int B, int Hkv, int rows, int Lk, int *out);
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, bool calib,
                           int nt, cudaStream_t stream);

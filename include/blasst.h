@@ -84,8 +84,9 @@ typedef struct blasst_opts {
     int block_n;               /* 0, or the fixed block size (128 prefill, 64 decode) */
     int num_splits;            /* decode: KV chunks per sequence; 0 -> 16 (d = 128) or 2
                                   (MLA, d = 576); -1 -> adaptive for d = 128
-                                  (blasst_decode_pick_splits with this device's SM count;
-                                  MLA rejects it with BLASST_ERR_INVALID) */
+                                  (blasst_decode_pick_splits_rows with the tile's rows
+                                  G * Lq and this device's SM count; MLA rejects it
+                                  with BLASST_ERR_INVALID) */
     int mode;                  /* blasst_calibrate only: 0 = prefill tiling, 1 = decode tiling */
     long long k_row_stride;    /* elements between consecutive keys; 0 -> d */
     long long v_row_stride;    /* elements between consecutive values; 0 -> dv */
@@ -307,6 +308,17 @@ BLASST_API blasst_status blasst_decode_noalloc(const void *q, const void *k, con
  * explicitly (the skip mask depends on the split count).  Size a caller
  * workspace with it too.  Invalid sizes return 1. */
 BLASST_API int blasst_decode_pick_splits(int B, int Hkv, int Lk, int num_sms);
+
+/* Host only.  The split count that num_splits = -1 selects for a tile of rows
+ * = G * Lq query rows: blasst_decode_pick_splits for tiles of up to 16 rows;
+ * for wider tiles (the tcgen05 kernel, two CTAs per SM) floor(4 * num_sms /
+ * (B * Hkv)) -- the most splits that keep the grid within two full waves of
+ * two CTAs per SM -- under the same cap (at least 32 blocks of 64 keys per
+ * split, at most 64) and at least 1.  Measured on B200 for 128 query heads on
+ * one KV head, batch 64, 32K keys (dense ms): 8 splits 0.214, 9 splits 0.208
+ * (this rule), 10 splits 0.253, 12 splits 0.233, 16 splits 0.237; past two
+ * waves the last one runs partly empty.  Invalid sizes return 1. */
+BLASST_API int blasst_decode_pick_splits_rows(int B, int Hkv, int rows, int Lk, int num_sms);
 
 BLASST_API size_t blasst_decode_workspace_bytes(int B, int Hq, int Lq, int dv, int num_splits);
 

@@ -189,6 +189,22 @@ def test_pick_splits(bl):
     assert f(0, 8, 100, 148) == 1 and f(1, 8, 100, 0) == 1
 
 
+def test_pick_splits_wide_tiles(bl):
+    f = bl.lib().blasst_decode_pick_splits_rows
+    narrow = bl.lib().blasst_decode_pick_splits
+    for B, Hkv, rows in ((32, 8, 4), (1, 8, 16), (4, 2, 1)):   # tiles of up to 16 rows: the narrow rule
+        assert f(B, Hkv, rows, 32768, 148) == narrow(B, Hkv, 32768, 148)
+    assert f(64, 1, 128, 32768, 148) == 9     # floor(4 * 148 / 64): 576 CTAs, under two waves of two per SM
+    assert f(32, 1, 128, 32768, 148) == 16    # floor(592 / 32) = 18, capped at 32 blocks per split
+    assert f(256, 1, 128, 32768, 148) == 2
+    assert f(1024, 1, 64, 32768, 148) == 1    # the batch fills two waves by itself
+    assert f(8, 1, 17, 2047, 148) == 1        # short cache: one split
+    for B in (1, 3, 16, 64, 200):
+        want = 4 * 132 // (B * 2)
+        assert f(B, 2, 32, 65536, 132) == max(1, min(min(64, 1024 // 32), want))
+    assert f(0, 1, 128, 100, 148) == 1 and f(1, 1, 128, 100, 0) == 1
+
+
 def test_adaptive_splits_only_where_supported(bl):
     mla = dict(num_splits=-1, dv=512, k_row_stride=576, v_row_stride=576)
     assert _call(bl, "blasst_decode", d=576, opts=bl.Opts(**mla)) == 1   # MLA

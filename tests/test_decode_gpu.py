@@ -366,3 +366,17 @@ def test_decode_adaptive_splits(bl):
     torch.cuda.synchronize()
     assert all(torch.equal(x, y) for x, y in zip(a, b))
     check_decode(bl, inp, 0.05, False, S)
+
+
+def test_decode_adaptive_splits_wide_tile(bl):
+    # a 64-row tile takes the wide rule (floor(4 * SMs / (B * Hkv)) under the cap); -1 equals that count
+    inp = planted_decode(4, 64, 1, 64 * 300 + 5, 128, seed=30, reading="blk")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    S = bl.decode_pick_splits(4, 1, 64 * 300 + 5, rows=64)
+    assert S == max(1, min(64, 300 // 32, 4 * sms // 4))
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    a = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=-1)
+    b = bl.decode(q, k, v, scale=inp.scale, lam=0.05, num_splits=S)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    check_decode(bl, inp, 0.05, False, S)

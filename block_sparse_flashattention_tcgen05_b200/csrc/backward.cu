@@ -78,13 +78,16 @@ constexpr int kTileBytes = 128 * 128 * 2;  // 128 rows x 128 bf16
 constexpr int kBoxBytes = kTileBytes / 2;  // 128 rows x 64 bf16 (one 128-byte swizzle box)
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusSmemAlign = 4;
-// CTA order: chunks of kOrderChunk consecutive KV blocks, one KV head after another within
-// a chunk, chunks in block order.  Blocks with more query tiles (causal: small j) still
-// start first, and the CTAs resident together mostly share one or two KV heads, so their
-// Q, dO tiles and dQ accumulator rows are reused in L2 (32K causal GQA: DRAM traffic per
-// launch 19.8 -> 8.1 GB dense and 30.6 -> 22.7 GB at 75 %, against the KV head as the
-// fastest index).
+// CTA order for long sequences (at least kOrderMinBlocks KV blocks): chunks of kOrderChunk
+// consecutive KV blocks, one KV head after another within a chunk, chunks in block order.
+// Blocks with more query tiles (causal: small j) still start early, and the CTAs resident
+// together mostly share one or two KV heads, so their Q, dO tiles and dQ accumulator rows
+// are reused in L2 (32K causal GQA: DRAM traffic per launch 19.8 -> 8.1 GB dense and
+// 30.6 -> 22.7 GB at 75 %).  Shorter sequences keep the KV head as the fastest index: there
+// a chunk is a large share of the blocks, and the longest CTAs of the last heads would
+// start too late (16K: 16 % slower with chunks of 64).
 constexpr int kOrderChunk = 64;
+constexpr int kOrderMinBlocks = 256;
 
 struct BwdTail {
     float nl2[2][128];  // per stage: -lse * log2(e) of the pair's 128 query rows
@@ -162,10 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     int j, hkv;
     {
-        const int q = blockIdx.x / (kOrderChunk * p.Hkv), r = blockIdx.x % (kOrderChunk * p.Hkv);
-        const int cq = min(kOrderChunk, p.nb - q * kOrderChunk);  // blocks in this chunk
+        const int chunk = p.nb >= kOrderMinBlocks ? kOrderChunk : 1;
+        const int q = blockIdx.x / (chunk * p.Hkv), r = blockIdx.x % (chunk * p.Hkv);
+        const int cq = min(chunk, p.nb - q * chunk);  // blocks in this chunk
         hkv = r / cq;
-        j = q * kOrderChunk + r % cq;
+        j = q * chunk + r % cq;
     }
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

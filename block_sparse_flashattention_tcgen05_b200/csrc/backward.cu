@@ -98,7 +98,10 @@ struct BwdTail {
     uint64_t kv_full;
     uint64_t qdo_full[2], qdo_empty[2];
     uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
-    uint64_t dq_staged;      // the compute warps have written dQ(t)'s rows to pair t's Q and dO stages
+    // [stage]: the compute warps have written dQ(t)'s rows to pair t's Q and dO stages.  One
+    // barrier per stage: the compute warps may stage pair t+1 before the reduce warp has seen
+    // pair t's phase, but pair t+2 (the same stage) only after the stage came back (stage_free).
+    uint64_t dq_staged[2];
     uint64_t stage_free[2];  // [stage]: the bulk reduce of dQ(t) has read the staged rows
     uint32_t tmem_base;
     int abort;
@@ -189,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&tl->dq_full, 1);
         mbar_init(&tl->dq_free, kComputeWarps);
         mbar_init(&tl->acc_done, 1);
-        mbar_init(&tl->dq_staged, kComputeWarps);
+        mbar_init(&tl->dq_staged[0], kComputeWarps);
+        mbar_init(&tl->dq_staged[1], kComputeWarps);
         mbar_init(&tl->stage_free[0], 1);
         mbar_init(&tl->stage_free[1], 1);
         tl->abort = 0;
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int i = first_tile(p, j), g = 0, t = 0;
             while (!tl->abort && next_pair(p, b, hkv, j, i, g)) {
                 const int st = t & 1;
-                if (!mbar_wait(&tl->dq_staged, t & 1, &tl->abort)) {
+                if (!mbar_wait(&tl->dq_staged[st], (t >> 1) & 1, &tl->abort)) {
                     set_timeout(tl, p.status);
                     break;
                 }
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < kCW; c++) stg[c * 128] = __uint_as_float(qa[c]);
             fence_proxy_async();  // the stores -> visible to the bulk copy's reads
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tl->dq_staged);
+            if (lane == 0) mbar_arrive(&tl->dq_staged[st]);
             t++;
             advance(p, i, g);
         }

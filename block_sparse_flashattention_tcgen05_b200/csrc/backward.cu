@@ -43,10 +43,10 @@
 // then, once dS^T(t) is ready: dQ^T(t), dK(t), dV(t), S(t+1).  Operations
 // issued by one thread execute in issue order, so S(t+1) overwrites P^T(t) only
 // after dV(t) has read it, and a commit covers every earlier operation.
-// dQ staging: once dK(t) and dV(t) have completed, pair t's Q and dO stages
-// are not read again, and they take dQ(t) as fp32 rows (queries 0-63 in the Q
-// stage, 64-127 in the dO stage, 512 bytes of head dims per row, the
-// accumulator's own layout) while the tensor core runs S(t+1).  The reduce
+// dQ staging: pair t's Q stage is not read again once dK(t) has completed, nor
+// its dO stage once dV(t) has, and they take dQ(t) as fp32 rows (queries 0-63
+// in the Q stage while the tensor core runs dV(t), 64-127 in the dO stage while
+// it runs S(t+1); 512 bytes of head dims per row, the accumulator's own layout).  The reduce
 // warp adds both ranges to the accumulator and hands the stages back to the
 // producer for pair t+2 (stage_free) once the bulk copies have read them.
 // Nothing on the compute warps' path waits for the reduction (staging in the
@@ -103,6 +103,7 @@ struct BwdTail {
     // pair t's phase, but pair t+2 (the same stage) only after the stage came back (stage_free).
     uint64_t dq_staged[2];
     uint64_t stage_free[2];  // [stage]: the bulk reduce of dQ(t) has read the staged rows
+    uint64_t dk_done;        // dK(t) has completed: pair t's Q stage takes dQ(t)'s rows 0-63
     uint32_t tmem_base;
     int abort;
 };
@@ -192,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&tl->dq_full, 1);
         mbar_init(&tl->dq_free, kComputeWarps);
         mbar_init(&tl->acc_done, 1);
+        mbar_init(&tl->dk_done, 1);
         mbar_init(&tl->dq_staged[0], kComputeWarps);
         mbar_init(&tl->dq_staged[1], kComputeWarps);
         mbar_init(&tl->stage_free[0], 1);
@@ -321,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < 8; kk++)
                     umma_ss2(tmem + 384, ds_km + koff(kk), q_mn + st * kStage16 + kk * (2048 >> 4), dhi, idesc_kmn,
                              (t > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&tl->dk_done);  // pair t's Q stage: free for dQ(t)'s rows 0-63
                 // dV += P^T dO (K = 128 queries; P^T of each column group in its own S^T columns)
 #pragma unroll
                 for (int kk = 0; kk < 8; kk++)
@@ -470,14 +473,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tl->dq_free);
-            // stage dQ(t) once dK(t) and dV(t) are done: query rows of 128 fp32 head dims, rows
-            // 0-63 in pair t's Q stage and 64-127 in its dO stage (a warp store covers 128
-            // contiguous bytes of one row); rows past Lq hold zeros (their P, hence dS, is 0)
-            if (!warp_wait(&tl->qdo_empty[st], (t >> 1) & 1, &tl->abort)) {
+            // stage dQ(t): query rows of 128 fp32 head dims (a warp store covers 128 contiguous
+            // bytes of one row), rows 0-63 in pair t's Q stage once dK(t) is done, rows 64-127 in
+            // its dO stage once dV(t) is done, so that half of the stores overlap dV(t); rows
+            // past Lq hold zeros (their P, hence dS, is 0)
+            const bool low_rows = hh * kCW < 64;
+            if (!(low_rows ? warp_wait(&tl->dk_done, t & 1, &tl->abort)
+                           : warp_wait(&tl->qdo_empty[st], (t >> 1) & 1, &tl->abort))) {
                 set_timeout(tl, p.status);
                 break;
             }
-            float *stg = reinterpret_cast<float *>(hh * kCW < 64 ? sQ + st * kTileBytes : sdO + st * kTileBytes) +
+            float *stg = reinterpret_cast<float *>(low_rows ? sQ + st * kTileBytes : sdO + st * kTileBytes) +
                          ((hh * kCW) & 63) * 128 + r;
 #pragma unroll
             for (int c = 0; c < kCW; c++) stg[c * 128] = __uint_as_float(qa[c]);

@@ -202,6 +202,50 @@ def test_backward_full_size_sampled_rows_and_invariants(bl):
         assert np.all(np.abs(dvh[hk].sum(axis=0) - want) <= 2.0 ** -6 * tot_v)
 
 
+def test_backward_long_sequence_partial_last_chunk(bl):
+    """261 KV blocks (33408 keys): the launch orders CTAs in chunks of 64 KV blocks, the last chunk
+    holding 5. Sampled dq rows against the oracle (rows seeing the last blocks included) and the key
+    sums sum_k dK_k = 0 and sum_k dV_k = sum of the group's dO rows, which miss a block whose CTA was
+    left out or run twice; the last block's dK and dV rows are nonzero."""
+    L = 261 * 128
+    inp = planted_prefill(1, 8, 2, L, 128, seed=71, reading="blk")
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    o, lse, mask, cnt = bl.prefill(q, k, v, scale=inp.scale, lam=0.0128, causal=True)
+    do_bits = upstream_grad(1, 8, L, 128, seed=10)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv = bl.prefill_backward(q, k, v, o, lse, to_dev(do_bits), scale=inp.scale, causal=True,
+                                     skip_mask=mask, status_word=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    bits = unpack_mask(mask.cpu().numpy(), L // 128)
+    rows = [(0, 0, 5), (0, 3, 20000), (0, 4, L - 300), (0, 7, L - 1)]
+    ref = oracle.backward_dq_rows(inp.q, inp.k, inp.v, do_bits, rows, scale=inp.scale, causal=True, skip=bits,
+                                  terms=True)
+    dqh = dq.float().cpu().numpy()
+    Kf = bf16_to_f32(inp.k).astype(np.float64)[0]
+    Vf = bf16_to_f32(inp.v).astype(np.float64)[0]
+    Dof = bf16_to_f32(do_bits).astype(np.float64)[0]
+    for n, (b, h, r) in enumerate(rows):
+        # the per-element bound of the 32K test: bf16 dS, the forward's bf16 O in D, the bf16 output
+        kk, vv = Kf[h // 4], Vf[h // 4]
+        p_, ds_, o_ = ref["P"][n], ref["dS"][n], ref["O"][n]
+        dD = (np.abs(Dof[h, r]) * (2.0 ** -8 * (p_ @ np.abs(vv)) + 2.0 ** -9 * np.abs(o_))).sum()
+        bound = (2.0 ** -9 * (np.abs(ref["dq"][n]) + inp.scale * (np.abs(ds_) @ np.abs(kk))) +
+                 inp.scale * dD * (p_ @ np.abs(kk)))
+        err = np.abs(dqh[b, h, r] - ref["dq"][n])
+        assert np.all(err <= bound + 1e-7), f"row {(b, h, r)}: worst {np.max(err / (bound + 1e-7)):.2f} of bound"
+    dkh = dk.double().cpu().numpy()[0]
+    dvh = dv.double().cpu().numpy()[0]
+    dov = torch.from_numpy(do_bits.view(np.int16)).view(torch.bfloat16).double().numpy()[0]
+    for hk in range(2):
+        tot = np.abs(dkh[hk]).sum(axis=0)
+        assert np.all(np.abs(dkh[hk].sum(axis=0)) <= 2.0 ** -6 * tot)
+        want = dov[hk * 4:(hk + 1) * 4].sum(axis=(0, 1))
+        tot_v = np.abs(dvh[hk]).sum(axis=0)
+        assert np.all(np.abs(dvh[hk].sum(axis=0) - want) <= 2.0 ** -6 * tot_v)
+        assert np.abs(dvh[hk, L - 128:]).sum() > 0 and np.abs(dkh[hk, L - 128:]).sum() > 0
+
+
 def test_backward_noncausal_more_queries_than_keys(bl):
     inp = random_normal(1, 4, 2, 500, 200, 128, seed=68)
     check_backward(bl, inp, 0.0, False, seed=8)

@@ -267,6 +267,19 @@ def test_seeded_mask_equals_prefix_max_closed_form(lam, splits):
     assert np.array_equal(r["skip"], skip)
 
 
+@pytest.mark.parametrize("splits", [3, 8])
+def test_seeded_mask_equals_prefix_max_closed_form_wide_tile(splits):
+    # a 64-row tile (64 query heads on one KV head, the shape of the tcgen05 decode): every row's
+    # prefix max, block 0 included, must allow the skip
+    inp = planted_decode(1, 64, 1, 2048, 32, seed=19, reading="blk")
+    for lam in (0.05, 0.3, 0.9):
+        r = _run(inp, lam, False, is_decode=True, num_splits=splits, BN=64, seed_splits=True)
+        skip, vis = closed_form_decisions(inp.q, inp.k, inp.scale, False, lam, 128, 64, is_decode=True,
+                                          num_splits=splits, seed_splits=True)
+        assert np.array_equal(r["visited"], vis)
+        assert np.array_equal(r["skip"], skip)
+
+
 def test_seeded_outputs_equal_masked_softmax():
     # block 0 enters later splits only through its maxima, never through l or O
     inp = planted_decode(1, 4, 1, 2048, 32, seed=4, reading="blk")
